@@ -1,0 +1,253 @@
+/*
+ * mfsdp.h - C ABI of the MatrixFSDP owner-local optimizer step on B200 (sm_100a).
+ *
+ * Method: "MatrixFSDP: communication-free matrix optimizers under ZeRO-3
+ * parameter sharding" (arxivlens summary page, Abstract; gist.science French
+ * and Portuguese technical summaries, Methodologie / Metodologia sections 1-2).
+ * Under owner-shaped ZeRO-3 placement each 2D weight lives whole on one
+ * data-parallel owner, so after the ordinary backward reduction the owner holds
+ * the full gradient and runs the Muon update locally with no collective;
+ * non-matrix tensors are packed into a tail that stays on AdamW.  This library
+ * is that owner-local step, plus the host-side owner planner.
+ *
+ * Conventions shared by every entry point
+ *  - Every call returns an int status: MFSDP_OK (0) or a negative MFSDP_ERR_*.
+ *    No C++ exception crosses the ABI.  mfsdp_status_string() names a status.
+ *  - Matrices are row-major, torch Linear layout: rows = out, cols = in.
+ *  - Device pointers are plain CUDA device addresses on the current device;
+ *    host pointers are ordinary host memory.  The caller owns every buffer;
+ *    the library allocates no device memory and keeps no state across calls
+ *    apart from a host-side cache of the descriptor table it last wrote into
+ *    a given workspace (see mfsdp_muon_step).
+ *  - "stream" is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  GPU work is enqueued asynchronously on it; arguments are
+ *    validated synchronously before anything is enqueued, and an invalid call
+ *    enqueues nothing.  Errors raised by kernels while they run are recorded
+ *    in a device status word read by mfsdp_get_device_status().
+ *  - A size of zero (n == 0, rows == 0 or cols == 0) is a no-op, not an error.
+ */
+#ifndef MFSDP_H
+#define MFSDP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+#define MFSDP_OK                        0
+#define MFSDP_ERR_INVALID_ARG          -1  /* NULL pointer, negative size, bad enum, aliasing */
+#define MFSDP_ERR_UNSUPPORTED_DTYPE    -2  /* dtype/mode combination not implemented */
+#define MFSDP_ERR_MISALIGNED           -3  /* pointer not aligned to its element size / 256 B workspace */
+#define MFSDP_ERR_WORKSPACE_TOO_SMALL  -4  /* workspace_bytes below mfsdp_muon_workspace_size() */
+#define MFSDP_ERR_CUDA                 -5  /* a CUDA runtime call failed (launch, copy, attribute) */
+#define MFSDP_ERR_TIMEOUT              -6  /* a bounded device-side wait gave up */
+#define MFSDP_ERR_DEVICE_FAULT         -7  /* a kernel detected an out-of-range index and skipped it */
+#define MFSDP_ERR_UNSUPPORTED_DEVICE   -8  /* current device is not sm_100 */
+
+/* ---- enums ----------------------------------------------------------- */
+#define MFSDP_DTYPE_F32   0
+#define MFSDP_DTYPE_BF16  1
+
+#define MFSDP_KIND_MATRIX 0   /* 2D weight: Muon on its owner */
+#define MFSDP_KIND_TAIL   1   /* non-matrix tensor: packed tail, AdamW */
+
+#define MFSDP_MODE_FP32   0   /* Newton-Schulz GEMMs in fp32 on FFMA (no tf32) */
+#define MFSDP_MODE_BF16   1   /* GEMM operands rounded to bf16, fp32 accumulate (tcgen05) */
+
+/* ---- planner ----------------------------------------------------------
+ * Passage: arxivlens summary page, Abstract (MatrixShard metadata, a
+ * balance-aware owner planner, one owner per 2D weight with empty shards
+ * elsewhere, non-matrix tensors packed into tail owners); gist.science French
+ * summary, Methodologie section 2, "Metadonnees MatrixShard & Planificateur
+ * Global" (owners balance resident bytes and optimizer work).
+ */
+typedef struct {
+    int64_t rows;     /* >= 0; a 1D tensor of length L is rows = L, cols = 1 */
+    int64_t cols;     /* >= 0 */
+    int32_t kind;     /* MFSDP_KIND_MATRIX or MFSDP_KIND_TAIL */
+    int32_t dtype;    /* MFSDP_DTYPE_* of a matrix's param and grad (tails are fp32) */
+} mfsdp_param_desc;
+
+/* One MatrixShard record: where a parameter lives and what it costs. */
+typedef struct {
+    int64_t param_id;        /* index into the planner's input array */
+    int64_t rows, cols;
+    int32_t owner;           /* owning rank in [0, world_size) */
+    int32_t kind;            /* MFSDP_KIND_* */
+    int32_t transposed;      /* 1 if rows > cols: Newton-Schulz runs on the transpose */
+    int32_t reserved;
+    double  ns_flops;        /* ns_steps * (4 r^2 c + 2 r^3), r = min, c = max; 0 for tails */
+    int64_t resident_bytes;  /* param + grad + fp32 momentum (matrix) or 16 B/elem (tail) */
+    int64_t owner_offset;    /* element offset in the owner's local buffer (matrices, id order)
+                                or in the packed tail (tail tensors, id order) */
+    double  shape_scale;     /* sqrt(max(1, rows / cols)); 1 for tails */
+} mfsdp_matrix_shard;
+
+/*
+ * mfsdp_plan - assign an owner to every parameter (host only, no CUDA call).
+ *   params          host array of n descriptors (read only)
+ *   n               number of parameters, >= 0
+ *   world_size      number of data-parallel ranks, >= 1
+ *   ns_steps        Newton-Schulz iteration count used in the FLOP cost, >= 0
+ *   out_shards      host array of n records, written (input order)
+ *   out_rank_flops  host array of world_size doubles, written (may be NULL)
+ *   out_rank_bytes  host array of world_size int64s, written (may be NULL)
+ * Rule: matrices sorted by (-ns_flops, -resident_bytes, id); each goes to the
+ * rank minimising (max((F_r+f)/Fbar, (B_r+b)/Bbar), F_r+f, rank); the whole
+ * tail is one unit placed last on the rank with the fewest bytes.
+ * Pure and deterministic.  Errors: MFSDP_ERR_INVALID_ARG.
+ */
+int mfsdp_plan(const mfsdp_param_desc* params, int64_t n, int32_t world_size, int32_t ns_steps,
+               mfsdp_matrix_shard* out_shards, double* out_rank_flops, int64_t* out_rank_bytes);
+
+/* The heaviest rank: largest FLOPs, then largest bytes, then lowest id. */
+int mfsdp_heaviest_rank(const double* rank_flops, const int64_t* rank_bytes, int32_t world_size,
+                        int32_t* out_rank);
+
+/* ---- Muon step --------------------------------------------------------
+ * Passage: arxivlens summary page, Abstract (Muon orthogonalises
+ * momentum-smoothed matrix updates with Newton-Schulz; the owner holds the
+ * whole matrix, so Newton-Schulz runs locally); gist.science French summary,
+ * Methodologie section 1 (the full gradient lands on the owner, which updates
+ * with zero optimizer-step communication).  Arithmetic per matrix (fp32
+ * unless stated):
+ *   buf <- beta buf + (1-beta) G ;  M <- (1-beta) G + beta buf   (nesterov = 1)
+ *                                   M <- buf                      (nesterov = 0)
+ *   X <- (rows > cols ? M^T : M) / (||M||_F + eps)        (X is r x c, r <= c)
+ *   ns_steps times:  A = X X^T ;  B = b A + c A A ;  X <- a X + B X
+ *   O = (transpose back) X * sqrt(max(1, rows/cols))
+ *   W <- W (1 - lr wd) - lr O        (one round-to-nearest-even store to W's dtype)
+ * MFSDP_MODE_BF16 rounds the GEMM operands (X, A, B) to bf16 and accumulates
+ * in fp32; the master X, A in the b A term and every epilogue stay fp32.
+ */
+typedef struct {
+    void*       param;       /* device, rows x cols, param_dtype; updated in place */
+    const void* grad;        /* device, rows x cols, grad_dtype; read only */
+    float*      momentum;    /* device, rows x cols fp32 momentum buffer; updated in place */
+    float*      update_out;  /* device, rows x cols fp32, optional (NULL = skip): receives O */
+    int64_t     rows, cols;  /* >= 0 */
+    int32_t     param_dtype; /* MFSDP_DTYPE_F32 or MFSDP_DTYPE_BF16 */
+    int32_t     grad_dtype;  /* MFSDP_DTYPE_F32 or MFSDP_DTYPE_BF16 */
+} mfsdp_matrix;
+
+typedef struct {
+    float   lr;              /* learning rate */
+    float   beta;            /* momentum coefficient in [0, 1) */
+    float   weight_decay;    /* decoupled, multiplied by lr */
+    float   eps;             /* added to the Frobenius norm (1e-7) */
+    float   a, b, c;         /* quintic coefficients (3.4445, -4.7750, 2.0315) */
+    int32_t ns_steps;        /* Newton-Schulz iterations, 0..16 (5) */
+    int32_t nesterov;        /* 1 = Nesterov, 0 = plain momentum */
+    int32_t mode;            /* MFSDP_MODE_FP32 or MFSDP_MODE_BF16 */
+} mfsdp_muon_hparams;
+
+/*
+ * mfsdp_muon_workspace_size - bytes of device workspace mfsdp_muon_step needs
+ * for this matrix list and mode (host only).  *bytes is written.
+ * Errors: MFSDP_ERR_INVALID_ARG, MFSDP_ERR_UNSUPPORTED_DTYPE.
+ */
+int mfsdp_muon_workspace_size(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
+                              size_t* bytes);
+
+/*
+ * mfsdp_muon_step - the owner's grouped Muon step over n matrices.
+ *   mats             host array of n matrix records (read during the call only)
+ *   hp               host pointer to the hyper-parameters
+ *   workspace        device, >= mfsdp_muon_workspace_size() bytes, 256-byte aligned,
+ *                    owned by the caller, dedicated to this matrix list: its head
+ *                    holds a descriptor table the library writes on the first call
+ *                    for a given (list, workspace) pair and reuses while the list
+ *                    is unchanged.  Calls that share a workspace must not overlap
+ *                    on the GPU.  Call mfsdp_muon_forget_workspace() before giving
+ *                    the memory another use.
+ *   stream           cudaStream_t as void*
+ * Alignment: param/grad aligned to their element size, momentum and
+ * update_out to 4 bytes (16-byte alignment enables vector access).  Matrices
+ * must not alias one another.  Launches: one momentum kernel, one norm kernel,
+ * three GEMM-phase kernels per Newton-Schulz iteration (the last also writes W),
+ * or one write kernel when ns_steps = 0.
+ * Errors: MFSDP_ERR_INVALID_ARG, MFSDP_ERR_UNSUPPORTED_DTYPE, MFSDP_ERR_MISALIGNED,
+ * MFSDP_ERR_WORKSPACE_TOO_SMALL, MFSDP_ERR_UNSUPPORTED_DEVICE, MFSDP_ERR_CUDA.
+ */
+int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Number of kernel launches one mfsdp_muon_step call with these arguments enqueues. */
+int mfsdp_muon_step_launches(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
+                             int32_t* launches);
+
+/* Drop the host-side cache entry for a workspace (before reusing its memory). */
+int mfsdp_muon_forget_workspace(void* workspace);
+
+/* ---- AdamW tail -------------------------------------------------------
+ * Passage: arxivlens summary page, Abstract (non-matrix tensors are packed
+ * into tail owners and stay on AdamW); gist.science French summary,
+ * Methodologie section 1, "Tenseurs Non-Matrices".
+ *   m <- beta1 m + (1-beta1) g ;  v <- beta2 v + (1-beta2) g^2
+ *   p <- p (1 - lr wd) - lr (m / (1-beta1^t)) / (sqrt(v / (1-beta2^t)) + eps)
+ */
+typedef struct {
+    float   lr, beta1, beta2, eps, weight_decay;
+    int32_t reserved;
+    int64_t step;            /* t >= 1, the step being taken */
+} mfsdp_adamw_hparams;
+
+/*
+ * mfsdp_adamw_tail - AdamW over a flat packed fp32 tail of n elements.
+ *   p, m, v  device fp32, updated in place;  g  device fp32, read only.
+ *   All four 4-byte aligned, non-overlapping (16-byte alignment enables
+ *   128-bit access).  Errors: MFSDP_ERR_INVALID_ARG, MFSDP_ERR_MISALIGNED,
+ *   MFSDP_ERR_UNSUPPORTED_DEVICE, MFSDP_ERR_CUDA.
+ */
+int mfsdp_adamw_tail(float* p, const float* g, float* m, float* v, int64_t n,
+                     const mfsdp_adamw_hparams* hp, void* stream);
+
+/* ---- profiling ---------------------------------------------------------
+ * Per-kernel-class CUDA-event timing of the library's own launches, for the
+ * benchmark's roofline figures.  Between mfsdp_profile_begin() and
+ * mfsdp_profile_end() every kernel the library launches (from any thread) is
+ * bracketed by two cudaEventRecord calls on its launch stream, up to
+ * max_launches launches; the rest run untimed.  mfsdp_profile_end()
+ * synchronises those events, sums durations per class and stops recording.
+ */
+#define MFSDP_KCLASS_MOMENTUM  0   /* momentum + layout + norm partials */
+#define MFSDP_KCLASS_NORM      1   /* Frobenius norm finalisation */
+#define MFSDP_KCLASS_GRAM      2   /* A = X X^T */
+#define MFSDP_KCLASS_POLY      3   /* B = b A + c A A */
+#define MFSDP_KCLASS_APPLY     4   /* X <- a X + B X (and the final write) */
+#define MFSDP_KCLASS_WRITE0    5   /* parameter write when ns_steps = 0 */
+#define MFSDP_KCLASS_ADAMW     6   /* AdamW tail */
+#define MFSDP_KCLASS_COUNT     8
+
+typedef struct {
+    int32_t launches[MFSDP_KCLASS_COUNT];  /* timed launches per class */
+    double  ms[MFSDP_KCLASS_COUNT];        /* summed device time per class, milliseconds */
+} mfsdp_profile;
+
+/* Start recording (max_launches >= 1 event pairs).  Errors: MFSDP_ERR_INVALID_ARG
+ * (already recording or max_launches < 1), MFSDP_ERR_CUDA. */
+int mfsdp_profile_begin(int32_t max_launches);
+
+/* Stop recording and fill *out.  Errors: MFSDP_ERR_INVALID_ARG (not recording), MFSDP_ERR_CUDA. */
+int mfsdp_profile_end(mfsdp_profile* out);
+
+/* ---- status ------------------------------------------------------------ */
+
+/* Synchronise `stream` and read (then clear) the device status word of the
+ * current device: MFSDP_OK or the first MFSDP_ERR_* a kernel recorded. */
+int mfsdp_get_device_status(void* stream, int32_t* status);
+
+/* Static text for a status code (never NULL). */
+const char* mfsdp_status_string(int32_t status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t mfsdp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MFSDP_H */

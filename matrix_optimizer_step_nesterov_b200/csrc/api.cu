@@ -1,0 +1,416 @@
+// C ABI entry points of libmfsdp: argument validation, the workspace layout,
+// the grouped tile tables and the launch sequence of the owner-local step.
+//
+// Step (per matrix, grouped over the owner's matrix list): "MatrixFSDP:
+// communication-free matrix optimizers under ZeRO-3 parameter sharding",
+// arxivlens summary page, Abstract -- the owner holds the whole matrix and
+// runs Muon's momentum + Newton-Schulz update locally; the tail stays on AdamW.
+#include "../../include/mfsdp.h"
+#include "internal.h"
+#include "gemm_tc.h"
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+#include <vector>
+
+namespace mfsdp {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
+
+int check_device() {
+    static int cached[64] = {0};  // 0 unknown, 1 ok, -1 unsupported
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MFSDP_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return MFSDP_ERR_UNSUPPORTED_DEVICE;
+    if (cached[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return MFSDP_ERR_CUDA;
+        }
+        cached[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    return cached[dev] == 1 ? MFSDP_OK : MFSDP_ERR_UNSUPPORTED_DEVICE;
+}
+
+bool aligned(const void* p, size_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }
+
+int validate_hparams(const mfsdp_muon_hparams* hp) {
+    if (!hp) return MFSDP_ERR_INVALID_ARG;
+    if (hp->mode != MFSDP_MODE_FP32 && hp->mode != MFSDP_MODE_BF16) return MFSDP_ERR_INVALID_ARG;
+    if (hp->ns_steps < 0 || hp->ns_steps > 16) return MFSDP_ERR_INVALID_ARG;
+    if (hp->nesterov != 0 && hp->nesterov != 1) return MFSDP_ERR_INVALID_ARG;
+    if (!std::isfinite(hp->lr) || !std::isfinite(hp->beta) || !std::isfinite(hp->weight_decay) ||
+        !std::isfinite(hp->eps) || !std::isfinite(hp->a) || !std::isfinite(hp->b) || !std::isfinite(hp->c))
+        return MFSDP_ERR_INVALID_ARG;
+    if (hp->eps < 0.f) return MFSDP_ERR_INVALID_ARG;
+    return MFSDP_OK;
+}
+
+int validate_matrix(const mfsdp_matrix& m) {
+    if (m.rows < 0 || m.cols < 0) return MFSDP_ERR_INVALID_ARG;
+    if (m.rows > (1LL << 30) || m.cols > (1LL << 30)) return MFSDP_ERR_INVALID_ARG;
+    if (m.param_dtype != MFSDP_DTYPE_F32 && m.param_dtype != MFSDP_DTYPE_BF16) return MFSDP_ERR_UNSUPPORTED_DTYPE;
+    if (m.grad_dtype != MFSDP_DTYPE_F32 && m.grad_dtype != MFSDP_DTYPE_BF16) return MFSDP_ERR_UNSUPPORTED_DTYPE;
+    if (m.rows == 0 || m.cols == 0) return MFSDP_OK;
+    if (!m.param || !m.grad || !m.momentum) return MFSDP_ERR_INVALID_ARG;
+    if (!aligned(m.param, m.param_dtype == MFSDP_DTYPE_BF16 ? 2 : 4)) return MFSDP_ERR_MISALIGNED;
+    if (!aligned(m.grad, m.grad_dtype == MFSDP_DTYPE_BF16 ? 2 : 4)) return MFSDP_ERR_MISALIGNED;
+    if (!aligned(m.momentum, 4)) return MFSDP_ERR_MISALIGNED;
+    if (m.update_out && !aligned(m.update_out, 4)) return MFSDP_ERR_MISALIGNED;
+    return MFSDP_OK;
+}
+
+// [begin, end) byte ranges of every user buffer, to reject aliasing between matrices
+int check_no_alias(const mfsdp_matrix* mats, int32_t n) {
+    struct Range { uintptr_t b, e; int32_t owner; bool writable; };
+    std::vector<Range> rs;
+    rs.reserve(static_cast<size_t>(n) * 4);
+    for (int32_t i = 0; i < n; ++i) {
+        const mfsdp_matrix& m = mats[i];
+        if (m.rows == 0 || m.cols == 0) continue;
+        const uintptr_t numel = static_cast<uintptr_t>(m.rows * m.cols);
+        const uintptr_t pe = m.param_dtype == MFSDP_DTYPE_BF16 ? 2 : 4;
+        const uintptr_t ge = m.grad_dtype == MFSDP_DTYPE_BF16 ? 2 : 4;
+        rs.push_back({reinterpret_cast<uintptr_t>(m.param), reinterpret_cast<uintptr_t>(m.param) + numel * pe, i, true});
+        rs.push_back({reinterpret_cast<uintptr_t>(m.grad), reinterpret_cast<uintptr_t>(m.grad) + numel * ge, i, false});
+        rs.push_back({reinterpret_cast<uintptr_t>(m.momentum), reinterpret_cast<uintptr_t>(m.momentum) + numel * 4, i, true});
+        if (m.update_out)
+            rs.push_back({reinterpret_cast<uintptr_t>(m.update_out), reinterpret_cast<uintptr_t>(m.update_out) + numel * 4, i, true});
+    }
+    std::sort(rs.begin(), rs.end(), [](const Range& x, const Range& y) { return x.b < y.b; });
+    // any overlap that involves a written range is an error (two grads may share memory)
+    uintptr_t max_end_w = 0, max_end_any = 0;
+    for (const Range& r : rs) {
+        if (r.b < max_end_w) return MFSDP_ERR_INVALID_ARG;
+        if (r.writable && r.b < max_end_any) return MFSDP_ERR_INVALID_ARG;
+        max_end_any = std::max(max_end_any, r.e);
+        if (r.writable) max_end_w = std::max(max_end_w, r.e);
+    }
+    return MFSDP_OK;
+}
+
+// Which GEMM engine runs the Newton-Schulz phases for this call.
+enum class Engine { Simt, Tc };
+
+Engine pick_engine(const mfsdp_muon_hparams* hp) {
+    return hp->mode == MFSDP_MODE_BF16 && tc_available() ? Engine::Tc : Engine::Simt;
+}
+
+// Workspace plan: head (descriptor table, tile tables, partials, scales), then
+// per-matrix X / A / B buffers, every region 256-byte aligned.
+struct Layout {
+    std::vector<MatDev> mats;          // device records (workspace pointers filled if base given)
+    std::vector<TileDev> sym_tiles;    // PH_GRAM / PH_POLY
+    std::vector<TileDev> gen_tiles;    // PH_APPLY / PH_FINAL
+    int32_t mom_tiles = 0;
+    size_t off_mats = 0, off_sym = 0, off_gen = 0, off_partials = 0, off_s = 0, head_end = 0;
+    size_t total = 0;
+    Engine engine = Engine::Simt;
+};
+
+void build_tiles(Layout& L, Engine eng) {
+    L.sym_tiles.clear();
+    L.gen_tiles.clear();
+    if (eng == Engine::Tc) {
+        tc_build_tiles(L.mats, L.sym_tiles, L.gen_tiles);
+        return;
+    }
+    const int T = kSimtTile;
+    for (int32_t mi = 0; mi < static_cast<int32_t>(L.mats.size()); ++mi) {
+        const MatDev& m = L.mats[mi];
+        const int tr_ = (m.r + T - 1) / T, tc_ = (m.c + T - 1) / T;
+        for (int i = 0; i < tr_; ++i)
+            for (int j = i; j < tr_; ++j) L.sym_tiles.push_back({mi, i, j, (m.c + 7) / 8});
+        for (int i = 0; i < tr_; ++i)
+            for (int j = 0; j < tc_; ++j) L.gen_tiles.push_back({mi, i, j, (m.r + 7) / 8});
+    }
+}
+
+int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp, char* base, Layout& L) {
+    const bool bf16 = hp->mode == MFSDP_MODE_BF16;
+    L.engine = pick_engine(hp);
+    L.mats.clear();
+    int32_t tile0 = 0;
+    for (int32_t i = 0; i < n; ++i) {
+        const mfsdp_matrix& u = in[i];
+        if (u.rows == 0 || u.cols == 0) continue;
+        MatDev m{};
+        m.param = u.param;
+        m.grad = u.grad;
+        m.buf = u.momentum;
+        m.update_out = u.update_out;
+        m.rows = u.rows;
+        m.cols = u.cols;
+        m.tr = u.rows > u.cols ? 1 : 0;
+        m.r = static_cast<int32_t>(std::min(u.rows, u.cols));
+        m.c = static_cast<int32_t>(std::max(u.rows, u.cols));
+        m.ldx = round8(m.c);
+        m.lda = round8(m.r);
+        m.param_bf16 = u.param_dtype == MFSDP_DTYPE_BF16;
+        m.grad_bf16 = u.grad_dtype == MFSDP_DTYPE_BF16;
+        m.mom_tile0 = tile0;
+        m.mom_tiles_n = static_cast<int32_t>((u.cols + kMomTile - 1) / kMomTile);
+        const int64_t tiles = ((u.rows + kMomTile - 1) / kMomTile) * m.mom_tiles_n;
+        if (tile0 + tiles > (1LL << 31) - 1) return MFSDP_ERR_INVALID_ARG;
+        tile0 += static_cast<int32_t>(tiles);
+        m.mom_vec = (u.cols % 4 == 0) && aligned(u.momentum, 16) &&
+                    aligned(u.grad, u.grad_dtype == MFSDP_DTYPE_BF16 ? 8 : 16);
+        m.shape_scale = static_cast<float>(std::sqrt(std::max(1.0, static_cast<double>(u.rows) / u.cols)));
+        L.mats.push_back(m);
+    }
+    L.mom_tiles = tile0;
+    build_tiles(L, L.engine);
+    const size_t nm = L.mats.size();
+    size_t off = 0;
+    L.off_mats = off;      off = align_up(off + nm * sizeof(MatDev));
+    L.off_sym = off;       off = align_up(off + L.sym_tiles.size() * sizeof(TileDev));
+    L.off_gen = off;       off = align_up(off + L.gen_tiles.size() * sizeof(TileDev));
+    L.off_partials = off;  off = align_up(off + static_cast<size_t>(L.mom_tiles) * sizeof(float));
+    L.off_s = off;         off = align_up(off + nm * sizeof(float));
+    L.head_end = off;
+    for (MatDev& m : L.mats) {
+        const size_t x_elems = static_cast<size_t>(m.r) * m.ldx;
+        const size_t a_elems = static_cast<size_t>(m.r) * m.lda;
+        auto take = [&](size_t bytes) -> char* {
+            char* p = base ? base + off : nullptr;
+            off = align_up(off + bytes);
+            return p;
+        };
+        if (bf16) {
+            m.xf[0] = reinterpret_cast<float*>(take(x_elems * 4));
+            m.xf[1] = nullptr;
+            m.xb[0] = reinterpret_cast<__nv_bfloat16*>(take(x_elems * 2));
+            m.xb[1] = reinterpret_cast<__nv_bfloat16*>(take(x_elems * 2));
+            m.af = reinterpret_cast<float*>(take(a_elems * 4));
+            m.ab = reinterpret_cast<__nv_bfloat16*>(take(a_elems * 2));
+            m.bm = take(a_elems * 2);
+        } else {
+            m.xf[0] = reinterpret_cast<float*>(take(x_elems * 4));
+            m.xf[1] = reinterpret_cast<float*>(take(x_elems * 4));
+            m.xb[0] = m.xb[1] = nullptr;
+            m.af = reinterpret_cast<float*>(take(a_elems * 4));
+            m.ab = nullptr;
+            m.bm = take(a_elems * 4);
+        }
+    }
+    L.total = off;
+    return MFSDP_OK;
+}
+
+// host cache: the head bytes last uploaded into each workspace
+struct CacheEntry { int dev; std::vector<char> head; };
+std::mutex g_cache_mu;
+std::unordered_map<uintptr_t, CacheEntry> g_cache;
+
+int validate_all(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp) {
+    if (n < 0) return MFSDP_ERR_INVALID_ARG;
+    int st = validate_hparams(hp);
+    if (st) return st;
+    if (n > 0 && !mats) return MFSDP_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i) {
+        st = validate_matrix(mats[i]);
+        if (st) return st;
+    }
+    return check_no_alias(mats, n);
+}
+
+}  // namespace
+}  // namespace mfsdp
+
+using namespace mfsdp;
+
+extern "C" int mfsdp_muon_workspace_size(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
+                                         size_t* bytes) {
+    if (!bytes) return MFSDP_ERR_INVALID_ARG;
+    int st = validate_all(mats, n, hp);
+    if (st) return st;
+    Layout L;
+    st = build_layout(mats, n, hp, nullptr, L);
+    if (st) return st;
+    *bytes = L.mats.empty() ? 0 : L.total;
+    return MFSDP_OK;
+}
+
+extern "C" int mfsdp_muon_step_launches(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
+                                        int32_t* launches) {
+    if (!launches) return MFSDP_ERR_INVALID_ARG;
+    int st = validate_all(mats, n, hp);
+    if (st) return st;
+    int32_t live = 0;
+    for (int32_t i = 0; i < n; ++i) live += (mats[i].rows > 0 && mats[i].cols > 0);
+    *launches = live == 0 ? 0 : 2 + (hp->ns_steps == 0 ? 1 : 3 * hp->ns_steps);
+    return MFSDP_OK;
+}
+
+extern "C" int mfsdp_muon_forget_workspace(void* workspace) {
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    g_cache.erase(reinterpret_cast<uintptr_t>(workspace));
+    return MFSDP_OK;
+}
+
+extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    int st = validate_all(mats, n, hp);
+    if (st) return st;
+    int32_t live = 0;
+    for (int32_t i = 0; i < n; ++i) live += (mats[i].rows > 0 && mats[i].cols > 0);
+    if (live == 0) return MFSDP_OK;
+    st = check_device();
+    if (st) return st;
+    if (!workspace) return MFSDP_ERR_INVALID_ARG;
+    if (!aligned(workspace, kAlign)) return MFSDP_ERR_MISALIGNED;
+    Layout L;
+    char* base = static_cast<char*>(workspace);
+    st = build_layout(mats, n, hp, base, L);
+    if (st) return st;
+    if (workspace_bytes < L.total) return MFSDP_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    // head bytes: descriptor table and tile tables
+    std::vector<char> head(L.off_partials, 0);
+    std::memcpy(head.data() + L.off_mats, L.mats.data(), L.mats.size() * sizeof(MatDev));
+    if (!L.sym_tiles.empty())
+        std::memcpy(head.data() + L.off_sym, L.sym_tiles.data(), L.sym_tiles.size() * sizeof(TileDev));
+    if (!L.gen_tiles.empty())
+        std::memcpy(head.data() + L.off_gen, L.gen_tiles.data(), L.gen_tiles.size() * sizeof(TileDev));
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(g_cache_mu);
+        auto it = g_cache.find(reinterpret_cast<uintptr_t>(workspace));
+        const bool fresh = it != g_cache.end() && it->second.dev == dev && it->second.head == head;
+        if (!fresh) {
+            if (cudaMemcpyAsync(base, head.data(), head.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) {
+                cudaGetLastError();
+                g_cache.erase(reinterpret_cast<uintptr_t>(workspace));
+                return MFSDP_ERR_CUDA;
+            }
+            g_cache[reinterpret_cast<uintptr_t>(workspace)] = CacheEntry{dev, std::move(head)};
+        }
+    }
+    const MatDev* d_mats = reinterpret_cast<const MatDev*>(base + L.off_mats);
+    const TileDev* d_sym = reinterpret_cast<const TileDev*>(base + L.off_sym);
+    const TileDev* d_gen = reinterpret_cast<const TileDev*>(base + L.off_gen);
+    float* d_partials = reinterpret_cast<float*>(base + L.off_partials);
+    float* d_s = reinterpret_cast<float*>(base + L.off_s);
+    const int32_t nm = static_cast<int32_t>(L.mats.size());
+
+    StepScalars sc{};
+    sc.a = hp->a; sc.b = hp->b; sc.c = hp->c;
+    sc.lr = hp->lr;
+    sc.decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * hp->weight_decay);
+    sc.beta = hp->beta;
+    sc.eps = hp->eps;
+    sc.nesterov = hp->nesterov;
+    sc.bf16_mode = hp->mode == MFSDP_MODE_BF16;
+
+    int slot = prof_before(MFSDP_KCLASS_MOMENTUM, s);
+    cudaError_t e = launch_momentum(d_mats, nm, L.mom_tiles, sc, d_partials, s);
+    prof_after(slot, s);
+    if (e != cudaSuccess) return MFSDP_ERR_CUDA;
+    slot = prof_before(MFSDP_KCLASS_NORM, s);
+    e = launch_norm(d_mats, nm, d_partials, d_s, hp->eps, s);
+    prof_after(slot, s);
+    if (e != cudaSuccess) return MFSDP_ERR_CUDA;
+    if (hp->ns_steps == 0) {
+        slot = prof_before(MFSDP_KCLASS_WRITE0, s);
+        e = launch_write0(d_mats, nm, L.mom_tiles, sc, d_s, s);
+        prof_after(slot, s);
+        return e == cudaSuccess ? MFSDP_OK : MFSDP_ERR_CUDA;
+    }
+    const int32_t nsym = static_cast<int32_t>(L.sym_tiles.size());
+    const int32_t ngen = static_cast<int32_t>(L.gen_tiles.size());
+    auto gemm = [&](Phase ph, const TileDev* tiles, int32_t ntiles, int32_t it, int cls) {
+        const int sl = prof_before(cls, s);
+        const cudaError_t r = L.engine == Engine::Tc
+                                  ? launch_gemm_tc(ph, d_mats, nm, tiles, ntiles, it, sc, d_s, s)
+                                  : launch_gemm_simt(ph, d_mats, nm, tiles, ntiles, it, sc, d_s, s);
+        prof_after(sl, s);
+        return r;
+    };
+    for (int32_t it = 0; it < hp->ns_steps; ++it) {
+        const Phase last = (it == hp->ns_steps - 1) ? PH_FINAL : PH_APPLY;
+        e = gemm(PH_GRAM, d_sym, nsym, it, MFSDP_KCLASS_GRAM);
+        if (e == cudaSuccess) e = gemm(PH_POLY, d_sym, nsym, it, MFSDP_KCLASS_POLY);
+        if (e == cudaSuccess) e = gemm(last, d_gen, ngen, it, MFSDP_KCLASS_APPLY);
+        if (e != cudaSuccess) return MFSDP_ERR_CUDA;
+    }
+    return MFSDP_OK;
+}
+
+extern "C" int mfsdp_adamw_tail(float* p, const float* g, float* m, float* v, int64_t n,
+                                const mfsdp_adamw_hparams* hp, void* stream) {
+    if (!hp || n < 0) return MFSDP_ERR_INVALID_ARG;
+    if (hp->step < 1) return MFSDP_ERR_INVALID_ARG;
+    if (!std::isfinite(hp->lr) || !std::isfinite(hp->beta1) || !std::isfinite(hp->beta2) ||
+        !std::isfinite(hp->eps) || !std::isfinite(hp->weight_decay))
+        return MFSDP_ERR_INVALID_ARG;
+    if (hp->beta1 < 0.f || hp->beta1 >= 1.f || hp->beta2 < 0.f || hp->beta2 >= 1.f)
+        return MFSDP_ERR_INVALID_ARG;
+    if (n == 0) return MFSDP_OK;
+    if (!p || !g || !m || !v) return MFSDP_ERR_INVALID_ARG;
+    if (!aligned(p, 4) || !aligned(g, 4) || !aligned(m, 4) || !aligned(v, 4)) return MFSDP_ERR_MISALIGNED;
+    // the four buffers must not overlap
+    {
+        const uintptr_t len = static_cast<uintptr_t>(n) * 4;
+        const uintptr_t b[4] = {reinterpret_cast<uintptr_t>(p), reinterpret_cast<uintptr_t>(g),
+                                reinterpret_cast<uintptr_t>(m), reinterpret_cast<uintptr_t>(v)};
+        for (int i = 0; i < 4; ++i)
+            for (int j = i + 1; j < 4; ++j)
+                if (b[i] < b[j] + len && b[j] < b[i] + len) return MFSDP_ERR_INVALID_ARG;
+    }
+    int st = check_device();
+    if (st) return st;
+    const double t = static_cast<double>(hp->step);
+    const float bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(hp->beta1), t));
+    const float bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(hp->beta2), t));
+    const float decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * hp->weight_decay);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int slot = prof_before(MFSDP_KCLASS_ADAMW, s);
+    const cudaError_t e = launch_adamw(p, g, m, v, n, hp->lr, hp->beta1, hp->beta2, hp->eps, decay, bc1, bc2, s);
+    prof_after(slot, s);
+    return e == cudaSuccess ? MFSDP_OK : MFSDP_ERR_CUDA;
+}
+
+extern "C" int mfsdp_get_device_status(void* stream, int32_t* status) {
+    if (!status) return MFSDP_ERR_INVALID_ARG;
+    int32_t* d = device_status_ptr();
+    if (!d) return MFSDP_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) { cudaGetLastError(); return MFSDP_ERR_CUDA; }
+    if (cudaMemcpy(&h, d, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) { cudaGetLastError(); return MFSDP_ERR_CUDA; }
+    const int32_t zero = 0;
+    if (cudaMemcpy(d, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) { cudaGetLastError(); return MFSDP_ERR_CUDA; }
+    *status = h;
+    return MFSDP_OK;
+}
+
+extern "C" const char* mfsdp_status_string(int32_t status) {
+    switch (status) {
+        case MFSDP_OK: return "MFSDP_OK";
+        case MFSDP_ERR_INVALID_ARG: return "MFSDP_ERR_INVALID_ARG: invalid argument";
+        case MFSDP_ERR_UNSUPPORTED_DTYPE: return "MFSDP_ERR_UNSUPPORTED_DTYPE: unsupported dtype";
+        case MFSDP_ERR_MISALIGNED: return "MFSDP_ERR_MISALIGNED: misaligned pointer";
+        case MFSDP_ERR_WORKSPACE_TOO_SMALL: return "MFSDP_ERR_WORKSPACE_TOO_SMALL: workspace too small";
+        case MFSDP_ERR_CUDA: return "MFSDP_ERR_CUDA: CUDA runtime error";
+        case MFSDP_ERR_TIMEOUT: return "MFSDP_ERR_TIMEOUT: bounded device wait gave up";
+        case MFSDP_ERR_DEVICE_FAULT: return "MFSDP_ERR_DEVICE_FAULT: kernel skipped an out-of-range index";
+        case MFSDP_ERR_UNSUPPORTED_DEVICE: return "MFSDP_ERR_UNSUPPORTED_DEVICE: device is not sm_100";
+        default: return "unknown mfsdp status";
+    }
+}
+
+extern "C" int32_t mfsdp_version(void) { return 100; }

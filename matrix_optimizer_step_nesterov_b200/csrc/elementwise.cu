@@ -1,0 +1,314 @@
+// HBM-bound kernels of the owner step: Nesterov momentum with the Frobenius
+// partial sums and the short-side-first layout of X, the per-matrix norm
+// finalisation, the ns_steps = 0 parameter write, and AdamW over the packed
+// tail.  Method passages: arxivlens summary page of "MatrixFSDP", Abstract
+// (momentum-smoothed Muon update on the owner; tail on AdamW).
+#include "internal.h"
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace mfsdp {
+namespace {
+
+__device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float load_elem(const void* p, int64_t i, int bf16) {
+    return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i])
+                : static_cast<const float*>(p)[i];
+}
+
+// four consecutive elements at p[i..i+3]; i % 4 == 0 and the base aligned
+__device__ __forceinline__ float4 load4(const void* p, int64_t i, int bf16) {
+    if (bf16) {
+        uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p) + i);
+        __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162*>(&raw.x);
+        __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162*>(&raw.y);
+        float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+    return *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
+}
+
+__device__ __forceinline__ void store4_bf16(__nv_bfloat16* p, int64_t i, float4 v) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 raw;
+    raw.x = *reinterpret_cast<uint32_t*>(&lo);
+    raw.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p + i) = raw;
+}
+
+// index of the matrix owning momentum tile `tile` (largest i with mom_tile0 <= tile)
+__device__ __forceinline__ int find_matrix(const MatDev* mats, int nmats, int tile) {
+    int lo = 0, hi = nmats - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (mats[mid].mom_tile0 <= tile) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// deterministic block sum (fixed shuffle tree, fixed warp order)
+template <typename T>
+__device__ __forceinline__ T block_sum(T v, T* smem) {
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) smem[warp] = v;
+    __syncthreads();
+    T r = 0;
+    if (threadIdx.x == 0) {
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r += smem[w];
+    }
+    return r;  // valid in thread 0
+}
+
+// ---------------------------------------------------------------------------
+// K1: one 64 x 64 tile of M per block of 256 threads.
+//   buf <- beta buf + (1-beta) G ;  M <- (1-beta) G + beta buf  (or M <- buf)
+// writes buf, the fp32 master X (M, or M^T when rows > cols) and, in bf16
+// mode, its bf16 operand copy; each tile's sum of M^2 goes to partials[tile].
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
+                float* __restrict__ partials, int32_t* status) {
+    __shared__ float tileM[kMomTile][kMomTile + 1];
+    __shared__ float red[8];
+    const int tile = blockIdx.x;
+    const int mi = find_matrix(mats, nmats, tile);
+    const MatDev& md = mats[mi];
+    const int local = tile - md.mom_tile0;
+    const int64_t rows = md.rows, cols = md.cols;
+    const int64_t tiles_m = (rows + kMomTile - 1) / kMomTile;
+    const int ti = local / md.mom_tiles_n, tj = local % md.mom_tiles_n;
+    if (local < 0 || ti >= tiles_m) {  // cannot happen with a host-built table
+        record_status(status, -7);
+        return;
+    }
+    const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;
+    const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
+    const float beta = sc.beta, omb = 1.0f - sc.beta;
+    const int tr = md.tr, gbf = md.grad_bf16, bf16_mode = sc.bf16_mode;
+    float* __restrict__ xf = md.xf[0];
+    __nv_bfloat16* __restrict__ xb = md.xb[0];
+    const int64_t ldx = md.ldx;
+    float sumsq = 0.f;
+
+    if (full && md.mom_vec) {
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            const int row = v >> 4, col = (v & 15) * 4;
+            const int64_t idx = (i0 + row) * cols + j0 + col;
+            float4 b = *reinterpret_cast<const float4*>(md.buf + idx);
+            const float4 g = load4(md.grad, idx, gbf);
+            float4 m;
+            b.x = beta * b.x + omb * g.x;  b.y = beta * b.y + omb * g.y;
+            b.z = beta * b.z + omb * g.z;  b.w = beta * b.w + omb * g.w;
+            if (sc.nesterov) {
+                m.x = omb * g.x + beta * b.x;  m.y = omb * g.y + beta * b.y;
+                m.z = omb * g.z + beta * b.z;  m.w = omb * g.w + beta * b.w;
+            } else {
+                m = b;
+            }
+            *reinterpret_cast<float4*>(md.buf + idx) = b;
+            sumsq += m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
+            if (!tr) {
+                const int64_t xi = (i0 + row) * ldx + j0 + col;
+                *reinterpret_cast<float4*>(xf + xi) = m;
+                if (bf16_mode) store4_bf16(xb, xi, m);
+            } else {
+                tileM[row][col] = m.x; tileM[row][col + 1] = m.y;
+                tileM[row][col + 2] = m.z; tileM[row][col + 3] = m.w;
+            }
+        }
+    } else {
+        for (int e = 0; e < 16; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            const int row = v >> 6, col = v & 63;
+            const int64_t i = i0 + row, j = j0 + col;
+            if (i < rows && j < cols) {
+                const int64_t idx = i * cols + j;
+                const float g = load_elem(md.grad, idx, gbf);
+                const float b = beta * md.buf[idx] + omb * g;
+                const float m = sc.nesterov ? (omb * g + beta * b) : b;
+                md.buf[idx] = b;
+                sumsq += m * m;
+                if (!tr) {
+                    xf[i * ldx + j] = m;
+                    if (bf16_mode) xb[i * ldx + j] = __float2bfloat16_rn(m);
+                } else {
+                    tileM[row][col] = m;
+                }
+            }
+        }
+    }
+    if (tr) {
+        __syncthreads();
+        // X = M^T: X[j][i] = M[i][j]; consecutive threads write consecutive i.
+        for (int e = 0; e < 16; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            const int orow = v >> 6, ocol = v & 63;   // X row = M col, X col = M row
+            const int64_t xr = j0 + orow, xc = i0 + ocol;
+            if (xr < cols && xc < rows) {
+                const float m = tileM[ocol][orow];
+                xf[xr * ldx + xc] = m;
+                if (bf16_mode) xb[xr * ldx + xc] = __float2bfloat16_rn(m);
+            }
+        }
+    }
+    const float tot = block_sum(sumsq, red);
+    if (threadIdx.x == 0) partials[tile] = tot;
+}
+
+// K2: s = 1 / (||M||_F + eps) per matrix; fixed-order fp64 sum of the tile partials.
+__global__ void __launch_bounds__(256)
+norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict__ partials,
+            float* __restrict__ s_out, float eps) {
+    __shared__ double red[8];
+    const int mi = blockIdx.x;
+    if (mi >= nmats) return;
+    const MatDev& md = mats[mi];
+    const int64_t tiles = ((md.rows + kMomTile - 1) / kMomTile) * md.mom_tiles_n;
+    double acc = 0.0;
+    for (int64_t t = threadIdx.x; t < tiles; t += blockDim.x) acc += (double)partials[md.mom_tile0 + t];
+    const double tot = block_sum(acc, red);
+    if (threadIdx.x == 0) s_out[mi] = (float)(1.0 / (sqrt(tot) + (double)eps));
+}
+
+// ns_steps = 0: O = scale * s * M, W <- W decay - lr O (same tiling as K1).
+__global__ void __launch_bounds__(256)
+write0_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, const float* __restrict__ s) {
+    const int tile = blockIdx.x;
+    const int mi = find_matrix(mats, nmats, tile);
+    const MatDev& md = mats[mi];
+    const int local = tile - md.mom_tile0;
+    const int ti = local / md.mom_tiles_n, tj = local % md.mom_tiles_n;
+    const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;
+    const float f = md.shape_scale * s[mi];
+    for (int e = 0; e < 16; ++e) {
+        const int v = e * 256 + threadIdx.x;
+        const int64_t i = i0 + (v >> 6), j = j0 + (v & 63);
+        if (i >= md.rows || j >= md.cols) continue;
+        const float x = md.tr ? md.xf[0][j * md.ldx + i] : md.xf[0][i * md.ldx + j];
+        const float o = f * x;
+        const int64_t idx = i * md.cols + j;
+        if (md.update_out) md.update_out[idx] = o;
+        if (md.param_bf16) {
+            __nv_bfloat16* w = static_cast<__nv_bfloat16*>(md.param);
+            w[idx] = __float2bfloat16_rn(fmaf(-sc.lr, o, __bfloat162float(w[idx]) * sc.decay));
+        } else {
+            float* w = static_cast<float*>(md.param);
+            w[idx] = fmaf(-sc.lr, o, w[idx] * sc.decay);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K6: AdamW over the packed fp32 tail.  28 algorithmic bytes per element.
+// ---------------------------------------------------------------------------
+struct AdamScalars {
+    float lr, beta1, beta2, eps, decay, bc1, bc2;
+};
+
+__device__ __forceinline__ void adam_elem(float& p, float g, float& m, float& v, const AdamScalars& a) {
+    m = a.beta1 * m + (1.0f - a.beta1) * g;
+    v = a.beta2 * v + (1.0f - a.beta2) * (g * g);
+    const float mhat = m / a.bc1;
+    const float vhat = v / a.bc2;
+    p = p * a.decay - a.lr * mhat / (sqrtf(vhat) + a.eps);
+}
+
+__global__ void __launch_bounds__(256)
+adamw_vec_kernel(float4* __restrict__ p, const float4* __restrict__ g, float4* __restrict__ m,
+                 float4* __restrict__ v, int64_t n4, AdamScalars a) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += 2 * stride) {
+        const int64_t i2 = i + stride;
+        float4 P = p[i], G = __ldcs(g + i), M = m[i], V = v[i];
+        float4 P2, G2, M2, V2;
+        const bool two = i2 < n4;
+        if (two) { P2 = p[i2]; G2 = __ldcs(g + i2); M2 = m[i2]; V2 = v[i2]; }
+        adam_elem(P.x, G.x, M.x, V.x, a); adam_elem(P.y, G.y, M.y, V.y, a);
+        adam_elem(P.z, G.z, M.z, V.z, a); adam_elem(P.w, G.w, M.w, V.w, a);
+        p[i] = P; m[i] = M; v[i] = V;
+        if (two) {
+            adam_elem(P2.x, G2.x, M2.x, V2.x, a); adam_elem(P2.y, G2.y, M2.y, V2.y, a);
+            adam_elem(P2.z, G2.z, M2.z, V2.z, a); adam_elem(P2.w, G2.w, M2.w, V2.w, a);
+            p[i2] = P2; m[i2] = M2; v[i2] = V2;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256)
+adamw_scalar_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+                    float* __restrict__ v, int64_t n, AdamScalars a) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        float P = p[i], M = m[i], V = v[i];
+        adam_elem(P, g[i], M, V, a);
+        p[i] = P; m[i] = M; v[i] = V;
+    }
+}
+
+int sm_count() {
+    static int count = 0;
+    if (count == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+        if (count <= 0) count = 148;
+    }
+    return count;
+}
+
+}  // namespace
+
+cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_tiles,
+                            const StepScalars& sc, float* partials, cudaStream_t st) {
+    if (total_tiles <= 0) return cudaSuccess;
+    momentum_kernel<<<total_tiles, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
+    return cudaGetLastError();
+}
+
+cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partials,
+                        float* s_out, float eps, cudaStream_t st) {
+    if (nmats <= 0) return cudaSuccess;
+    norm_kernel<<<nmats, 256, 0, st>>>(d_mats, nmats, partials, s_out, eps);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_write0(const MatDev* d_mats, int32_t nmats, int32_t total_tiles,
+                          const StepScalars& sc, const float* s, cudaStream_t st) {
+    if (total_tiles <= 0) return cudaSuccess;
+    write0_kernel<<<total_tiles, 256, 0, st>>>(d_mats, nmats, sc, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, int64_t n,
+                         float lr, float beta1, float beta2, float eps, float decay,
+                         float bc1, float bc2, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    AdamScalars a{lr, beta1, beta2, eps, decay, bc1, bc2};
+    const bool vec = (n % 4 == 0) &&
+                     ((reinterpret_cast<uintptr_t>(p) | reinterpret_cast<uintptr_t>(g) |
+                       reinterpret_cast<uintptr_t>(m) | reinterpret_cast<uintptr_t>(v)) % 16 == 0);
+    const int64_t work = vec ? n / 4 : n;
+    int64_t blocks = (work + 2 * 256 - 1) / (2 * 256);
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    if (vec) {
+        adamw_vec_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+            reinterpret_cast<float4*>(p), reinterpret_cast<const float4*>(g),
+            reinterpret_cast<float4*>(m), reinterpret_cast<float4*>(v), work, a);
+    } else {
+        adamw_scalar_kernel<<<(unsigned)blocks, 256, 0, st>>>(p, g, m, v, n, a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace mfsdp

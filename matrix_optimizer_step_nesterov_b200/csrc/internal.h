@@ -1,0 +1,87 @@
+// Internal declarations shared by the host dispatcher and the kernels of
+// libmfsdp.  Nothing here crosses the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace mfsdp {
+
+// Per-matrix record the kernels read from the workspace head.  X is the
+// r x c working matrix (r <= c): M itself, or M^T when rows > cols.
+struct MatDev {
+    void*        param;       // W, rows x cols, param dtype
+    const void*  grad;        // G, rows x cols, grad dtype
+    float*       buf;         // momentum, rows x cols fp32
+    float*       update_out;  // optional O, rows x cols fp32
+    float*       xf[2];       // fp32 X: bf16 mode keeps one in-place master, fp32 mode ping-pongs
+    __nv_bfloat16* xb[2];     // bf16 X operands (bf16 mode), ping-pong
+    float*       af;          // fp32 A = X X^T (r x r)
+    __nv_bfloat16* ab;        // bf16 copy of A (bf16 mode)
+    void*        bm;          // B = b A + c A A: bf16 (bf16 mode) or fp32
+    int64_t      rows, cols;  // the parameter's own shape
+    int64_t      ldx;         // leading dimension (elements) of every X buffer
+    int64_t      lda;         // leading dimension (elements) of A and B buffers
+    int32_t      r, c;        // X shape
+    int32_t      tr;          // rows > cols
+    int32_t      param_bf16;
+    int32_t      grad_bf16;
+    int32_t      mom_tile0;   // first momentum tile of this matrix
+    int32_t      mom_tiles_n; // momentum tiles along cols
+    int32_t      mom_vec;     // 1: 16-byte vector access is legal for this matrix
+    float        shape_scale; // sqrt(max(1, rows/cols))
+    int32_t      pad_;
+};
+
+// One output tile of a grouped GEMM phase.
+struct TileDev {
+    int32_t mat;
+    int32_t tm;    // tile row index
+    int32_t tn;    // tile column index
+    int32_t kblk;  // K depth in units of the kernel's K block (scheduling weight)
+};
+
+enum Phase : int32_t {
+    PH_GRAM = 0,   // A = s^2 * X X^T          (symmetric, upper tiles, mirrored store)
+    PH_POLY = 1,   // B = b A + c * A A        (symmetric, upper tiles, mirrored store)
+    PH_APPLY = 2,  // X <- s * (a X + B X)
+    PH_FINAL = 3,  // last iteration: O = scale * s * (a X + B X); W <- W (1 - lr wd) - lr O
+};
+
+struct StepScalars {
+    float a, b, c;
+    float lr;
+    float decay;       // 1 - lr * wd
+    float beta;
+    float eps;
+    int32_t nesterov;
+    int32_t bf16_mode;
+};
+
+constexpr int kMomTile = 64;   // momentum kernel tile: 64 x 64 elements of M
+
+// launch timing hooks (profile.cu): slot = prof_before(class, stream); launch; prof_after(slot, stream)
+int prof_before(int cls, cudaStream_t s);
+void prof_after(int slot, cudaStream_t s);
+
+// device status word helpers (defined in status.cu)
+int32_t* device_status_ptr();   // device address of this device's status word (nullptr on error)
+
+// ---- launchers (return cudaError_t of the launch) ----
+cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_tiles,
+                            const StepScalars& sc, float* partials, cudaStream_t st);
+cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partials,
+                        float* s_out, float eps, cudaStream_t st);
+cudaError_t launch_write0(const MatDev* d_mats, int32_t nmats, int32_t total_tiles,
+                          const StepScalars& sc, const float* s, cudaStream_t st);
+cudaError_t launch_gemm_simt(Phase ph, const MatDev* d_mats, int32_t nmats, const TileDev* d_tiles, int32_t ntiles,
+                             int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st);
+cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, int64_t n,
+                         float lr, float beta1, float beta2, float eps, float decay,
+                         float bc1, float bc2, cudaStream_t st);
+
+constexpr int kSimtTile = 128;  // SIMT GEMM block tile (square)
+
+}  // namespace mfsdp

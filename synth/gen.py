@@ -115,6 +115,17 @@ def matrix_inputs(wl: Workload, spec: ParamSpec, step: int = 0,
     return MatrixInputs(spec, W, G, buf, sigma, rank)
 
 
+def matrix_inputs_many(wl: Workload, specs, step: int = 0, buf_init: str = "zeros",
+                       threads: Optional[int] = None):
+    """matrix_inputs for many matrices, drawn in parallel threads (same values
+    as drawing them one by one: every matrix has its own streams)."""
+    import concurrent.futures as cf
+    import os
+    n = threads or min(32, os.cpu_count() or 1)
+    with cf.ThreadPoolExecutor(max_workers=n) as ex:
+        return list(ex.map(lambda s: matrix_inputs(wl, s, step=step, buf_init=buf_init), specs))
+
+
 @dataclasses.dataclass
 class TailInputs:
     p: np.ndarray

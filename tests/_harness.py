@@ -1,0 +1,175 @@
+"""Test harness: seeded inputs -> (GPU path through the C ABI, fp64 oracle) -> metrics.
+
+The two sides share only the seeded inputs from ``synth``.  The GPU side goes
+through ``matrix_optimizer_step_nesterov_b200`` (libmfsdp); the oracle side
+through ``oracle``.  No expected value is ever taken from the GPU path except
+where a check is explicitly "given the GPU's own O" (the parameter-write
+check, which tests the write alone).
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import os
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+import torch
+
+import oracle
+from synth import workloads as W
+from synth.gen import matrix_inputs_many, tail_inputs
+
+TOL_O = {"fp32": 1e-4, "bf16": 2e-2}
+TOL_BUF = 1e-6
+TOL_ADAMW = 1e-6
+
+_TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def rel_frob(x: np.ndarray, ref: np.ndarray) -> float:
+    den = float(np.linalg.norm(ref))
+    num = float(np.linalg.norm(np.asarray(x, np.float64) - ref))
+    return num / den if den > 0 else num
+
+
+def ordered_bits(x: torch.Tensor) -> np.ndarray:
+    """Map float32 / bfloat16 values to integers whose difference counts ulps."""
+    if x.dtype == torch.bfloat16:
+        i = x.view(torch.int16).to(torch.int64).numpy()
+        return np.where(i < 0, -(i & 0x7FFF), i)
+    i = x.to(torch.float32).view(torch.int32).to(torch.int64).numpy()
+    return np.where(i < 0, -(i & 0x7FFFFFFF), i)
+
+
+def ulp_distance(a: torch.Tensor, b: torch.Tensor) -> np.ndarray:
+    return np.abs(ordered_bits(a) - ordered_bits(b))
+
+
+def owner_share(wl: W.Workload):
+    """The matrices a workload steps: all of them, or the heaviest planned rank's
+    (planned with the oracle's planner; the product planner is tested equal)."""
+    if wl.world_size is None:
+        return wl.matrices
+    entries, F, B = oracle.plan_owners(wl.params, wl.world_size)
+    h = oracle.heaviest_rank(F, B)
+    by_pid = {p.pid: p for p in wl.params}
+    return [by_pid[e.pid] for e in entries if e.owner == h and e.kind == W.MATRIX]
+
+
+@dataclasses.dataclass
+class HostState:
+    specs: List[W.ParamSpec]
+    W: List[np.ndarray]
+    G: List[np.ndarray]
+    buf: List[np.ndarray]
+
+
+def host_state(wl: W.Workload, specs: Sequence[W.ParamSpec], step: int = 0, buf_init: str = "zeros") -> HostState:
+    ins = matrix_inputs_many(wl, specs, step=step, buf_init=buf_init)
+    return HostState(list(specs), [i.W for i in ins], [i.G for i in ins], [i.buf for i in ins])
+
+
+@dataclasses.dataclass
+class GpuResult:
+    W: List[torch.Tensor]      # cpu tensors in the param dtype
+    O: List[Optional[np.ndarray]]
+    buf: List[np.ndarray]
+
+
+def gpu_step(hs: HostState, mode: str, want_o: Optional[Sequence[int]] = None, ns_steps: int = 5,
+             nesterov: bool = True, lr: float = 0.02, beta: float = 0.95, weight_decay: float = 0.01,
+             grads: Optional[List[np.ndarray]] = None, repeat: int = 1) -> GpuResult:
+    """Run the product step over every matrix of ``hs`` in ONE grouped call
+    (``repeat`` calls in a row with the same gradients)."""
+    from matrix_optimizer_step_nesterov_b200 import MuonOwnerStep
+    dev = torch.device("cuda")
+    want = set(range(len(hs.specs))) if want_o is None else set(want_o)
+    params, gs, bufs, outs = [], [], [], []
+    for k, s in enumerate(hs.specs):
+        dt = _TORCH_DT[s.dtype]
+        params.append(torch.from_numpy(hs.W[k]).to(dt).to(dev))
+        g = hs.G[k] if grads is None else grads[k]
+        gs.append(torch.from_numpy(g).to(dt).to(dev))
+        bufs.append(torch.from_numpy(hs.buf[k]).to(dev))
+        outs.append(torch.empty(s.rows, s.cols, dtype=torch.float32, device=dev) if k in want else None)
+    step = MuonOwnerStep(params, gs, bufs, outs, lr=lr, beta=beta, weight_decay=weight_decay,
+                         ns_steps=ns_steps, nesterov=nesterov, mode=mode)
+    for _ in range(repeat):
+        step.step()
+    torch.cuda.synchronize()
+    res = GpuResult([p.cpu() for p in params],
+                    [o.cpu().numpy().astype(np.float64) if o is not None else None for o in outs],
+                    [b.cpu().numpy() for b in bufs])
+    step.close()
+    del params, gs, bufs, outs
+    return res
+
+
+def oracle_step(hs: HostState, k: int, ns_steps: int = 5, nesterov: bool = True, lr: float = 0.02,
+                beta: float = 0.95, weight_decay: float = 0.01):
+    hp = oracle.MuonHParams(lr=lr, beta=beta, weight_decay=weight_decay, ns_steps=ns_steps, nesterov=nesterov)
+    return oracle.muon_step(hs.W[k].astype(np.float64), hs.G[k].astype(np.float64),
+                            hs.buf[k].astype(np.float64), hp)
+
+
+def check_write(W0: np.ndarray, O_gpu: np.ndarray, W_gpu: torch.Tensor, lr: float = 0.02,
+                wd: float = 0.01) -> int:
+    """Max ulp distance of the GPU's parameter write from the fp64 write of the
+    GPU's own O, rounded once to the parameter dtype."""
+    ref = W0.astype(np.float64) * (1.0 - lr * wd) - lr * O_gpu
+    ref_t = torch.from_numpy(ref).to(W_gpu.dtype)
+    return int(ulp_distance(W_gpu, ref_t).max()) if ref.size else 0
+
+
+def compare_matrix(hs: HostState, res: GpuResult, k: int, mode: str, **kw) -> Dict[str, float]:
+    Wn, O, bn = oracle_step(hs, k, **kw)
+    out = {"rel_O": rel_frob(res.O[k], O) if res.O[k] is not None else float("nan"),
+           "rel_buf": rel_frob(res.buf[k], bn)}
+    if res.O[k] is not None:
+        out["write_ulp"] = check_write(hs.W[k], res.O[k], res.W[k],
+                                       lr=kw.get("lr", 0.02), wd=kw.get("weight_decay", 0.01))
+    return out
+
+
+def assert_parity(metrics: Dict[str, float], mode: str, label: str = "") -> None:
+    assert metrics["rel_O"] <= TOL_O[mode], f"{label} rel Frobenius error of O {metrics['rel_O']:.3e} > {TOL_O[mode]}"
+    assert metrics["rel_buf"] <= TOL_BUF, f"{label} momentum rel error {metrics['rel_buf']:.3e}"
+    if "write_ulp" in metrics:
+        assert metrics["write_ulp"] <= 2, f"{label} parameter write off by {metrics['write_ulp']} ulp"
+
+
+# ---- AdamW ----------------------------------------------------------------------
+
+def adamw_tolerance_ok(x: np.ndarray, ref: np.ndarray) -> bool:
+    """|d| <= 1e-6 |ref| + 2^-23 max|ref| per element (the floor covers cancellation)."""
+    if ref.size == 0:
+        return True
+    d = np.abs(np.asarray(x, np.float64) - ref)
+    bound = TOL_ADAMW * np.abs(ref) + 2.0 ** -23 * float(np.max(np.abs(ref)))
+    return bool(np.all(d <= bound))
+
+
+def gpu_adamw(p, g, m, v, t, offset: int = 0, **hp):
+    from matrix_optimizer_step_nesterov_b200 import adamw_tail
+    dev = torch.device("cuda")
+    n = p.size
+
+    def up(x):
+        buf = torch.zeros(n + offset, dtype=torch.float32, device=dev)
+        buf[offset:] = torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev)
+        return buf, buf[offset:]
+
+    (_, P), (_, G), (_, M), (_, V) = up(p), up(g), up(m), up(v)
+    adamw_tail(P, G, M, V, t, **hp)
+    torch.cuda.synchronize()
+    return P.cpu().numpy(), M.cpu().numpy(), V.cpu().numpy()
+
+
+def gpu_available() -> bool:
+    return torch.cuda.is_available()
+
+
+def lib_built() -> bool:
+    from matrix_optimizer_step_nesterov_b200 import _lib
+    return os.path.exists(_lib.LIB_PATH)

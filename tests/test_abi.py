@@ -1,0 +1,182 @@
+"""Host-side checks of libmfsdp: it loads, exports every symbol include/mfsdp.h
+declares, validates arguments before touching the GPU, and its planner agrees
+exactly with the oracle planner.  No compute call runs here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from synth import workload
+from synth.workloads import custom_workload, MATRIX
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from matrix_optimizer_step_nesterov_b200 import build
+    build.build()
+    from matrix_optimizer_step_nesterov_b200 import _lib
+    return _lib
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mfsdp.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mfsdp_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names(lib):
+    assert declared_functions() == sorted(lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    cdll = ctypes.CDLL(lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(cdll, name), f"libmfsdp.so does not export {name}"
+
+
+def test_nm_shows_c_linkage(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True, text=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in syms
+
+
+def test_status_strings_and_version(lib):
+    assert lib.status_string(0) == "MFSDP_OK"
+    for code in range(-8, 0):
+        assert lib.status_string(code).startswith("MFSDP_ERR_")
+    assert lib.status_string(12345) == "unknown mfsdp status"
+    assert lib.mfsdp_version() == 100
+
+
+def _descs(wl):
+    return [(p.rows, p.cols, p.kind, 1 if p.dtype == "bf16" else 0) for p in wl.params]
+
+
+@pytest.mark.parametrize("name", ["tiny", "block", "7b_share", "32b_share", "skew"])
+def test_planner_matches_oracle_exactly(lib, name):
+    wl = workload(name)
+    R = wl.world_size or 4
+    shards, F, B = lib.mfsdp_plan(_descs(wl), R)
+    entries, Fo, Bo = oracle.plan_owners(wl.params, R)
+    assert [s.owner for s in shards] == [e.owner for e in entries]
+    assert [s.owner_offset for s in shards] == [e.owner_offset for e in entries]
+    assert [bool(s.transposed) for s in shards] == [e.transposed for e in entries]
+    assert [s.ns_flops for s in shards] == [e.ns_flops for e in entries]
+    assert [s.resident_bytes for s in shards] == [e.resident_bytes for e in entries]
+    assert [s.shape_scale for s in shards] == [e.shape_scale for e in entries]
+    assert F == Fo and B == Bo
+    assert lib.mfsdp_heaviest_rank(F, B) == oracle.heaviest_rank(Fo, Bo)
+
+
+def test_planner_rejects_bad_arguments(lib):
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_plan([(4, 4, 0, 1)], 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_plan([(-1, 4, 0, 1)], 2)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_plan([(4, 4, 0, 7)], 2)
+    assert e.value.status == lib.MFSDP_ERR_UNSUPPORTED_DTYPE
+    shards, F, B = lib.mfsdp_plan([], 3)
+    assert shards == [] and F == [0.0, 0.0, 0.0]
+
+
+def _mat(lib, rows, cols, base=1 << 20, pdt=1, gdt=1):
+    e = 2 if pdt == 1 else 4
+    n = rows * cols
+    return lib.Matrix(base, base + 4 * n + 4096, base + 8 * n + 8192, None, rows, cols, pdt, gdt)
+
+
+def test_workspace_size_is_host_only_and_grows_with_shapes(lib):
+    hp = lib.muon_hparams(mode=lib.MFSDP_MODE_BF16)
+    s1 = lib.mfsdp_muon_workspace_size([_mat(lib, 256, 512)], hp)
+    s2 = lib.mfsdp_muon_workspace_size([_mat(lib, 512, 256)], hp)
+    s3 = lib.mfsdp_muon_workspace_size([_mat(lib, 256, 1024)], hp)
+    assert s1 == s2 > 0 and s3 > s1
+    # r x c = 256 x 512: fp32 master + two bf16 operands + fp32 A + bf16 A + bf16 B
+    assert s1 >= 256 * 512 * (4 + 2 + 2) + 256 * 256 * (4 + 2 + 2)
+    hp32 = lib.muon_hparams(mode=lib.MFSDP_MODE_FP32)
+    assert lib.mfsdp_muon_workspace_size([_mat(lib, 256, 512, pdt=0, gdt=0)], hp32) >= 256 * 512 * 8 + 256 * 256 * 8
+    assert lib.mfsdp_muon_workspace_size([], hp) == 0
+    assert lib.mfsdp_muon_workspace_size([_mat(lib, 0, 512)], hp) == 0
+
+
+def test_step_validation_errors_precede_any_device_work(lib):
+    hp = lib.muon_hparams()
+    m = _mat(lib, 64, 64)
+    bad = lib.muon_hparams(ns_steps=17)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step([m], bad, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    bad = lib.muon_hparams(mode=5)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step([m], bad, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    bad = lib.muon_hparams(lr=float("nan"))
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step([m], bad, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    # misaligned bf16 param
+    mm = lib.Matrix(m.param + 1, m.grad, m.momentum, None, 64, 64, 1, 1)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step([mm], hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_MISALIGNED
+    # NULL grad
+    mm = lib.Matrix(m.param, None, m.momentum, None, 64, 64, 1, 1)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step([mm], hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    # unsupported dtype code
+    mm = lib.Matrix(m.param, m.grad, m.momentum, None, 64, 64, 9, 1)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step([mm], hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_UNSUPPORTED_DTYPE
+    # two matrices writing the same momentum buffer
+    m2 = lib.Matrix(m.param + (1 << 24), m.grad + (1 << 24), m.momentum, None, 64, 64, 1, 1)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step([m, m2], hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    # negative shape
+    mm = lib.Matrix(m.param, m.grad, m.momentum, None, -1, 64, 1, 1)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step([mm], hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+
+
+def test_empty_step_is_a_noop_without_a_device(lib):
+    hp = lib.muon_hparams()
+    lib.mfsdp_muon_step([], hp, 0, 0, 0)
+    lib.mfsdp_muon_step([_mat(lib, 0, 64)], hp, 0, 0, 0)
+
+
+def test_launch_count(lib):
+    hp = lib.muon_hparams()
+    assert lib.mfsdp_muon_step_launches([_mat(lib, 64, 64)], hp) == 2 + 3 * 5
+    assert lib.mfsdp_muon_step_launches([_mat(lib, 64, 64)], lib.muon_hparams(ns_steps=0)) == 3
+    assert lib.mfsdp_muon_step_launches([], hp) == 0
+
+
+def test_adamw_validation(lib):
+    hp = lib.adamw_hparams(step=0)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_adamw_tail(1 << 20, 2 << 20, 3 << 20, 4 << 20, 16, hp, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    hp = lib.adamw_hparams(step=1)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_adamw_tail((1 << 20) + 2, 2 << 20, 3 << 20, 4 << 20, 16, hp, 0)
+    assert e.value.status == lib.MFSDP_ERR_MISALIGNED
+    with pytest.raises(lib.MfsdpError) as e:   # p and m overlap
+        lib.mfsdp_adamw_tail(1 << 20, 2 << 20, (1 << 20) + 32, 4 << 20, 16, hp, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_adamw_tail(0, 2 << 20, 3 << 20, 4 << 20, 16, hp, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    lib.mfsdp_adamw_tail(0, 0, 0, 0, 0, hp, 0)   # n == 0 is a no-op
