@@ -196,6 +196,8 @@ int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp
             m.af = reinterpret_cast<float*>(take(a_elems * 4));
             m.ab = reinterpret_cast<__nv_bfloat16*>(take(a_elems * 2));
             m.bm = take(a_elems * 2);
+            m.da = reinterpret_cast<float*>(take(static_cast<size_t>(m.r) * 4));
+            m.db = reinterpret_cast<float*>(take(static_cast<size_t>(m.r) * 4));
         } else {
             m.xf[0] = reinterpret_cast<float*>(take(x_elems * 4));
             m.xf[1] = reinterpret_cast<float*>(take(x_elems * 4));
@@ -203,6 +205,8 @@ int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp
             m.af = reinterpret_cast<float*>(take(a_elems * 4));
             m.ab = nullptr;
             m.bm = take(a_elems * 4);
+            m.da = reinterpret_cast<float*>(take(static_cast<size_t>(m.r) * 4));
+            m.db = reinterpret_cast<float*>(take(static_cast<size_t>(m.r) * 4));
         }
     }
     L.total = off;

@@ -8,6 +8,8 @@
 //   PH_POLY   B = b A + c A A     upper-triangle tiles, mirrored store (A symmetric, so A A = A A^T)
 //   PH_APPLY  X <- s (a X + B X)
 //   PH_FINAL  O = scale s (a X + B X);  W <- W (1 - lr wd) - lr O
+// in the diagonal-split form of internal.h: the GEMM operands are the
+// zero-diagonal parts E_A, E_B; the diagonals d_A, d_B enter in fp32 epilogues.
 // s is the Frobenius scale 1/(||M||+eps) on the first iteration and 1 after:
 // the momentum kernel stores M unnormalised and the scale is folded here.
 #include "internal.h"
@@ -180,22 +182,38 @@ simt_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, int32_t nmats,
             if (ph == PH_GRAM) {
                 if (gi > gj) continue;
                 const float v = (sg * sg) * a;
-                md.af[(int64_t)gi * md.lda + gj] = v;
-                md.af[(int64_t)gj * md.lda + gi] = v;
-                if (BF16) {
-                    md.ab[(int64_t)gi * md.lda + gj] = __float2bfloat16_rn(v);
-                    md.ab[(int64_t)gj * md.lda + gi] = __float2bfloat16_rn(v);
+                if (gi == gj) {
+                    md.da[gi] = v;
+                    md.af[(int64_t)gi * md.lda + gi] = 0.f;
+                    if (BF16) md.ab[(int64_t)gi * md.lda + gi] = __float2bfloat16_rn(0.f);
+                } else {
+                    md.af[(int64_t)gi * md.lda + gj] = v;
+                    md.af[(int64_t)gj * md.lda + gi] = v;
+                    if (BF16) {
+                        md.ab[(int64_t)gi * md.lda + gj] = __float2bfloat16_rn(v);
+                        md.ab[(int64_t)gj * md.lda + gi] = __float2bfloat16_rn(v);
+                    }
                 }
             } else if (ph == PH_POLY) {
                 if (gi > gj) continue;
-                const float v = sc.b * md.af[(int64_t)gi * md.lda + gj] + sc.c * a;
                 T* bm = reinterpret_cast<T*>(md.bm);
-                store_val<T>(bm + (int64_t)gi * md.lda + gj, v);
-                store_val<T>(bm + (int64_t)gj * md.lda + gi, v);
+                const float di = md.da[gi];
+                if (gi == gj) {
+                    // A_ii = d_i, (A A)_ii = (E E)_ii + d_i^2
+                    const float v = sc.b * di + sc.c * fmaf(di, di, a);
+                    md.db[gi] = v;
+                    store_val<T>(bm + (int64_t)gi * md.lda + gi, 0.f);
+                } else {
+                    const float e = md.af[(int64_t)gi * md.lda + gj];
+                    const float a2 = fmaf(di + md.da[gj], e, a);
+                    const float v = sc.b * e + sc.c * a2;
+                    store_val<T>(bm + (int64_t)gi * md.lda + gj, v);
+                    store_val<T>(bm + (int64_t)gj * md.lda + gi, v);
+                }
             } else {
                 const int64_t xi = (int64_t)gi * md.ldx + gj;
                 const float xin = md.xf[BF16 ? 0 : cur][xi];
-                const float v = sg * (sc.a * xin + a);
+                const float v = sg * fmaf(sc.a + md.db[gi], xin, a);
                 if (ph == PH_APPLY) {
                     if (BF16) {
                         md.xf[0][xi] = v;

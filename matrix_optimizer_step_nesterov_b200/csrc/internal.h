@@ -18,9 +18,11 @@ struct MatDev {
     float*       update_out;  // optional O, rows x cols fp32
     float*       xf[2];       // fp32 X: bf16 mode keeps one in-place master, fp32 mode ping-pongs
     __nv_bfloat16* xb[2];     // bf16 X operands (bf16 mode), ping-pong
-    float*       af;          // fp32 A = X X^T (r x r)
-    __nv_bfloat16* ab;        // bf16 copy of A (bf16 mode)
-    void*        bm;          // B = b A + c A A: bf16 (bf16 mode) or fp32
+    float*       af;          // fp32 E_A = A - diag(A), A = X X^T (r x r, zero diagonal)
+    __nv_bfloat16* ab;        // bf16 copy of E_A (bf16 mode GEMM operand)
+    void*        bm;          // E_B = B - diag(B), B = b A + c A A: bf16 (bf16 mode) or fp32
+    float*       da;          // diag(A), r entries, fp32
+    float*       db;          // diag(B), r entries, fp32
     int64_t      rows, cols;  // the parameter's own shape
     int64_t      ldx;         // leading dimension (elements) of every X buffer
     int64_t      lda;         // leading dimension (elements) of A and B buffers
@@ -43,11 +45,18 @@ struct TileDev {
     int32_t kblk;  // K depth in units of the kernel's K block (scheduling weight)
 };
 
+// Diagonal-split form of one Newton-Schulz iteration.  With A = D_A + E_A and
+// B = D_B + E_B (D diagonal, E zero-diagonal), the GEMMs take only the
+// zero-diagonal parts as operands and the diagonals stay exact in fp32:
+//   A A = E_A E_A + (d_i + d_j) E_A,ij + d_i^2 delta_ij
+//   B X = E_B X + d_B,i X_ij
+// In bf16 mode this keeps the large diagonal terms (and the near-cancellation
+// a X + D_B X) out of bf16 rounding; the GEMM work is unchanged.
 enum Phase : int32_t {
-    PH_GRAM = 0,   // A = s^2 * X X^T          (symmetric, upper tiles, mirrored store)
-    PH_POLY = 1,   // B = b A + c * A A        (symmetric, upper tiles, mirrored store)
-    PH_APPLY = 2,  // X <- s * (a X + B X)
-    PH_FINAL = 3,  // last iteration: O = scale * s * (a X + B X); W <- W (1 - lr wd) - lr O
+    PH_GRAM = 0,   // A = s^2 X X^T -> E_A (fp32 + operand copy), d_A   (upper tiles, mirrored)
+    PH_POLY = 1,   // B = b A + c A A -> E_B operand, d_B                (upper tiles, mirrored)
+    PH_APPLY = 2,  // X <- s ((a + d_B,i) X + E_B X)
+    PH_FINAL = 3,  // last iteration: O = scale * X_new; W <- W (1 - lr wd) - lr O
 };
 
 struct StepScalars {
