@@ -112,19 +112,22 @@ Engine pick_engine(const mfsdp_muon_hparams* hp) {
 // per-matrix X / A / B buffers, every region 256-byte aligned.
 struct Layout {
     std::vector<MatDev> mats;          // device records (workspace pointers filled if base given)
-    std::vector<TileDev> sym_tiles;    // PH_GRAM / PH_POLY
+    std::vector<TileDev> sym_tiles;    // PH_GRAM
+    std::vector<TileDev> poly_tiles;   // PH_POLY
     std::vector<TileDev> gen_tiles;    // PH_APPLY / PH_FINAL
     int32_t mom_tiles = 0;
-    size_t off_mats = 0, off_sym = 0, off_gen = 0, off_partials = 0, off_s = 0, head_end = 0;
+    size_t off_mats = 0, off_maps = 0, off_sym = 0, off_poly = 0, off_gen = 0, off_partials = 0, off_s = 0;
+    size_t head_end = 0, maps_bytes = 0;
     size_t total = 0;
     Engine engine = Engine::Simt;
 };
 
 void build_tiles(Layout& L, Engine eng) {
     L.sym_tiles.clear();
+    L.poly_tiles.clear();
     L.gen_tiles.clear();
     if (eng == Engine::Tc) {
-        tc_build_tiles(L.mats, L.sym_tiles, L.gen_tiles);
+        tc_build_tiles(L.mats, L.sym_tiles, L.poly_tiles, L.gen_tiles);
         return;
     }
     const int T = kSimtTile;
@@ -136,6 +139,7 @@ void build_tiles(Layout& L, Engine eng) {
         for (int i = 0; i < tr_; ++i)
             for (int j = 0; j < tc_; ++j) L.gen_tiles.push_back({mi, i, j, (m.r + 7) / 8});
     }
+    L.poly_tiles = L.sym_tiles;
 }
 
 int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp, char* base, Layout& L) {
@@ -175,7 +179,10 @@ int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp
     const size_t nm = L.mats.size();
     size_t off = 0;
     L.off_mats = off;      off = align_up(off + nm * sizeof(MatDev));
+    L.maps_bytes = L.engine == Engine::Tc ? tc_maps_bytes(nm) : 0;
+    L.off_maps = off;      off = align_up(off + L.maps_bytes);
     L.off_sym = off;       off = align_up(off + L.sym_tiles.size() * sizeof(TileDev));
+    L.off_poly = off;      off = align_up(off + L.poly_tiles.size() * sizeof(TileDev));
     L.off_gen = off;       off = align_up(off + L.gen_tiles.size() * sizeof(TileDev));
     L.off_partials = off;  off = align_up(off + static_cast<size_t>(L.mom_tiles) * sizeof(float));
     L.off_s = off;         off = align_up(off + nm * sizeof(float));
@@ -285,8 +292,11 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     // head bytes: descriptor table and tile tables
     std::vector<char> head(L.off_partials, 0);
     std::memcpy(head.data() + L.off_mats, L.mats.data(), L.mats.size() * sizeof(MatDev));
+    if (L.maps_bytes && !tc_encode_maps(L.mats, head.data() + L.off_maps)) return MFSDP_ERR_CUDA;
     if (!L.sym_tiles.empty())
         std::memcpy(head.data() + L.off_sym, L.sym_tiles.data(), L.sym_tiles.size() * sizeof(TileDev));
+    if (!L.poly_tiles.empty())
+        std::memcpy(head.data() + L.off_poly, L.poly_tiles.data(), L.poly_tiles.size() * sizeof(TileDev));
     if (!L.gen_tiles.empty())
         std::memcpy(head.data() + L.off_gen, L.gen_tiles.data(), L.gen_tiles.size() * sizeof(TileDev));
     int dev = 0;
@@ -306,6 +316,8 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     }
     const MatDev* d_mats = reinterpret_cast<const MatDev*>(base + L.off_mats);
     const TileDev* d_sym = reinterpret_cast<const TileDev*>(base + L.off_sym);
+    const TileDev* d_poly = reinterpret_cast<const TileDev*>(base + L.off_poly);
+    const void* d_maps = base + L.off_maps;
     const TileDev* d_gen = reinterpret_cast<const TileDev*>(base + L.off_gen);
     float* d_partials = reinterpret_cast<float*>(base + L.off_partials);
     float* d_s = reinterpret_cast<float*>(base + L.off_s);
@@ -339,7 +351,7 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     auto gemm = [&](Phase ph, const TileDev* tiles, int32_t ntiles, int32_t it, int cls) {
         const int sl = prof_before(cls, s);
         const cudaError_t r = L.engine == Engine::Tc
-                                  ? launch_gemm_tc(ph, d_mats, nm, tiles, ntiles, it, sc, d_s, s)
+                                  ? launch_gemm_tc(ph, d_mats, d_maps, nm, tiles, ntiles, it, sc, d_s, s)
                                   : launch_gemm_simt(ph, d_mats, nm, tiles, ntiles, it, sc, d_s, s);
         prof_after(sl, s);
         return r;
@@ -347,7 +359,7 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     for (int32_t it = 0; it < hp->ns_steps; ++it) {
         const Phase last = (it == hp->ns_steps - 1) ? PH_FINAL : PH_APPLY;
         e = gemm(PH_GRAM, d_sym, nsym, it, MFSDP_KCLASS_GRAM);
-        if (e == cudaSuccess) e = gemm(PH_POLY, d_sym, nsym, it, MFSDP_KCLASS_POLY);
+        if (e == cudaSuccess) e = gemm(PH_POLY, d_poly, nsym, it, MFSDP_KCLASS_POLY);
         if (e == cudaSuccess) e = gemm(last, d_gen, ngen, it, MFSDP_KCLASS_APPLY);
         if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     }

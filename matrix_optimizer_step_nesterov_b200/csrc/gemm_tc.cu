@@ -182,7 +182,7 @@ __device__ __forceinline__ void epilogue_chunk(int ph, const MatDev& md, int ite
     const int cur = iter & 1, nxt = cur ^ 1;
     if (ph == PH_GRAM) {
         const float s2 = sg * sg;
-        #pragma unroll 4
+        #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int gj = gj0 + t;
             if (gj >= Ncols || gi > gj) continue;
@@ -201,7 +201,7 @@ __device__ __forceinline__ void epilogue_chunk(int ph, const MatDev& md, int ite
     } else if (ph == PH_POLY) {
         __nv_bfloat16* bm = static_cast<__nv_bfloat16*>(md.bm);
         const float di = md.da[gi];
-        #pragma unroll 4
+        #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int gj = gj0 + t;
             if (gj >= Ncols || gi > gj) continue;
@@ -221,7 +221,7 @@ __device__ __forceinline__ void epilogue_chunk(int ph, const MatDev& md, int ite
         float* xrow = md.xf[0] + (int64_t)gi * md.ldx;
         if (ph == PH_APPLY) {
             __nv_bfloat16* xbn = md.xb[nxt] + (int64_t)gi * md.ldx;
-            #pragma unroll 4
+            #pragma unroll
             for (int t = 0; t < 32; ++t) {
                 const int gj = gj0 + t;
                 if (gj >= Ncols) continue;
@@ -230,7 +230,7 @@ __device__ __forceinline__ void epilogue_chunk(int ph, const MatDev& md, int ite
                 store_bf16(xbn + gj, v);
             }
         } else {
-            #pragma unroll 4
+            #pragma unroll
             for (int t = 0; t < 32; ++t) {
                 const int gj = gj0 + t;
                 if (gj >= Ncols) continue;
@@ -260,13 +260,14 @@ tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __res
     // 1024-byte aligned stage ring (128 B swizzle atoms need 1024 B alignment)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    // bars: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+    // bars: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], mma_done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
     const uint32_t tfull0 = smem_u32(bars + 2 * STAGES), tempty0 = smem_u32(bars + 2 * STAGES + 2);
+    const uint32_t mma_done = smem_u32(bars + 2 * STAGES + 4);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -277,6 +278,7 @@ tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __res
             mbar_init(tfull0 + 8 * i, 1);
             mbar_init(tempty0 + 8 * i, 4);   // one arrive per epilogue warp
         }
+        mbar_init(mma_done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -299,6 +301,9 @@ tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __res
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            int issued[STAGES];                  // parity of the last fill issued per stage, -1 = none
+            #pragma unroll
+            for (int i = 0; i < STAGES; ++i) issued[i] = -1;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const TileDev td = tiles[t];
                 const MatDev& md = mats[td.mat];
@@ -323,14 +328,16 @@ tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __res
                         for (int q = 0; q < BN / 64; ++q)
                             tma_load_2d(sb + q * (BK * 128), bmap, fb, j0 + 64 * q, kb * BK);
                     }
+                    issued[stage] = static_cast<int>(phase);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok) {
-                // drain: wait (bounded) for every stage's last load so no copy lands after exit
+                // aborting: wait (bounded, 10 ms each) until every issued load has landed
                 for (int i = 0; i < STAGES; ++i) {
+                    if (issued[i] < 0) continue;
                     const unsigned long long t0 = globaltimer();
-                    while (!mbar_try_wait(full0 + 8 * i, 0) && !mbar_try_wait(full0 + 8 * i, 1) &&
+                    while (!mbar_try_wait(full0 + 8 * i, static_cast<uint32_t>(issued[i])) &&
                            globaltimer() - t0 < 10000000ull) {
                     }
                 }
@@ -371,6 +378,11 @@ tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __res
                 if (!ok) break;
                 tc_commit(tfull0 + 8 * acc);           // accumulator ready for the epilogue
                 if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+            // every MMA this thread issued has completed before TMEM is freed (bounded)
+            tc_commit(mma_done);
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(mma_done, 0) && globaltimer() - t0 < 100000000ull) {
             }
         }
     } else {
