@@ -182,6 +182,25 @@ int mfsdp_muon_step_launches(const mfsdp_matrix* mats, int32_t n, const mfsdp_mu
 /* Drop the host-side cache entry for a workspace (before reusing its memory). */
 int mfsdp_muon_forget_workspace(void* workspace);
 
+/*
+ * mfsdp_muon_step_noalloc - mfsdp_muon_step without a caller workspace, for
+ * callers that cannot allocate device memory at step time: code running under
+ * CUDA stream capture, hosts that hand out every byte from their own
+ * pre-planned pools, loops that must not enter an allocator.  The paper has no
+ * counterpart; this is a deployment convenience of this library.
+ *   mats, n, hp, stream  as for mfsdp_muon_step (same validation, same result)
+ * Scratch: a fixed 64 MiB array compiled into the library, one per GPU that
+ * loads it, held until process exit.  Lists whose mfsdp_muon_workspace_size()
+ * exceeds 64 MiB are rejected with MFSDP_ERR_WORKSPACE_TOO_SMALL before any
+ * GPU work.  The call allocates no device memory.
+ * The first call on a device resolves the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call shares the one array, so calls that
+ * overlap on the GPU (other streams, other threads) race; serialise them.
+ * Nothing in the array needs to start at zero: each call writes what it reads.
+ */
+int mfsdp_muon_step_noalloc(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp, void* stream);
+
 /* ---- AdamW tail -------------------------------------------------------
  * Passage: arxivlens summary page, Abstract (non-matrix tensors are packed
  * into tail owners and stay on AdamW); gist.science French summary,

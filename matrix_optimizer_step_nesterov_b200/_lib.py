@@ -37,7 +37,7 @@ EXPORTED = (
     "mfsdp_plan", "mfsdp_heaviest_rank", "mfsdp_muon_workspace_size", "mfsdp_muon_step",
     "mfsdp_muon_step_launches", "mfsdp_muon_forget_workspace", "mfsdp_adamw_tail",
     "mfsdp_get_device_status", "mfsdp_status_string", "mfsdp_version",
-    "mfsdp_profile_begin", "mfsdp_profile_end",
+    "mfsdp_profile_begin", "mfsdp_profile_end", "mfsdp_muon_step_noalloc",
 )
 
 KCLASS_NAMES = ("momentum", "norm", "gram", "poly", "apply", "write0", "adamw", "unused")
@@ -124,6 +124,8 @@ def load() -> ctypes.CDLL:
     lib.mfsdp_profile_begin.restype = ctypes.c_int
     lib.mfsdp_profile_end.argtypes = [ctypes.POINTER(Profile)]
     lib.mfsdp_profile_end.restype = ctypes.c_int
+    lib.mfsdp_muon_step_noalloc.argtypes = [ctypes.POINTER(Matrix), i32, ctypes.POINTER(MuonHParams), p]
+    lib.mfsdp_muon_step_noalloc.restype = ctypes.c_int
     lib.mfsdp_version.argtypes = []
     lib.mfsdp_version.restype = ctypes.c_int32
     _lib = lib
@@ -239,3 +241,16 @@ def mfsdp_profile_end() -> dict:
     _check(load().mfsdp_profile_end(ctypes.byref(out)), "mfsdp_profile_end")
     return {KCLASS_NAMES[k]: (int(out.launches[k]), float(out.ms[k]))
             for k in range(8) if out.launches[k] > 0}
+
+
+# ---- step without a caller workspace ----------------------------------------------------
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def mfsdp_muon_step_noalloc(mats: Sequence[Matrix], hp: MuonHParams, stream: int) -> None:
+    """mfsdp_muon_step with the library's fixed 64 MiB device scratch: for callers
+    that cannot allocate device memory (stream capture, host-managed memory pools).
+    Calls that overlap on the GPU share the scratch and race."""
+    _check(load().mfsdp_muon_step_noalloc(matrix_array(mats), len(mats), ctypes.byref(hp), stream),
+           "mfsdp_muon_step_noalloc")
