@@ -75,6 +75,20 @@ def ns_flops_dense(specs, steps: int = 5) -> float:
     return tot
 
 
+def split_groups(specs, n_groups: int) -> List[List[int]]:
+    """Contiguous groups of matrix indices with about equal dense NS FLOPs."""
+    costs = [ns_flops_dense([s]) for s in specs]
+    total = sum(costs)
+    groups: List[List[int]] = [[] for _ in range(n_groups)]
+    acc, g = 0.0, 0
+    for i, c in enumerate(costs):
+        if g < n_groups - 1 and groups[g] and acc + c / 2 > total * (g + 1) / n_groups:
+            g += 1
+        groups[g].append(i)
+        acc += c
+    return [grp for grp in groups if grp]
+
+
 def max_over_ranks(x: float) -> float:
     import torch
     import torch.distributed as dist
@@ -294,7 +308,10 @@ def run_ours(args) -> int:
     ms_local = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms_local)
 
-    # e2e through host buffers: grads in (pinned H2D), updated params out (D2H)
+    # e2e through host buffers: every gradient in (pinned H2D) and every updated
+    # parameter out (D2H) each step.  The owner's matrices are split into
+    # --e2e-groups groups stepped one after another through the same C ABI, so
+    # that the copies of one group overlap the step of another.
     e2e = None
     if not args.no_e2e:
         hG = [g.cpu().pin_memory() for g in Gs]
@@ -304,17 +321,38 @@ def run_ours(args) -> int:
             htp = torch.empty(tp.shape, dtype=tp.dtype, pin_memory=True)
         h2d = sum(g.numel() * g.element_size() for g in hG) + (htg.numel() * 4 if tail_n else 0)
         d2h = sum(w.numel() * w.element_size() for w in hW) + (htp.numel() * 4 if tail_n else 0)
+        groups = split_groups(specs, max(1, min(args.e2e_groups, len(specs))))
+        gsteps = [MuonOwnerStep([Ws[i] for i in grp], [Gs[i] for i in grp], [Bs[i] for i in grp], mode=args.mode)
+                  for grp in groups]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
         def e2e_step():
-            for d, h in zip(Gs, hG):
-                d.copy_(h, non_blocking=True)
-            if tail_n:
-                tg.copy_(htg, non_blocking=True)
-            one_step()
-            for h, d in zip(hW, Ws):
-                h.copy_(d, non_blocking=True)
-            if tail_n:
-                htp.copy_(tp, non_blocking=True)
+            s_in.wait_stream(stream)                 # the previous step no longer reads the grads
+            ev_in = []
+            with torch.cuda.stream(s_in):
+                for g, grp in enumerate(groups):
+                    for i in grp:
+                        Gs[i].copy_(hG[i], non_blocking=True)
+                    if g == 0 and tail_n:
+                        tg.copy_(htg, non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(s_in)
+                    ev_in.append(ev)
+            for g, grp in enumerate(groups):
+                stream.wait_event(ev_in[g])
+                gsteps[g].step(stream)
+                if g == 0 and tail_n:
+                    t_counter[0] += 1
+                    adamw_tail(tp, tg, tm, tv, t_counter[0], stream=stream)
+                ev = torch.cuda.Event()
+                ev.record(stream)
+                s_out.wait_event(ev)
+                with torch.cuda.stream(s_out):
+                    for i in grp:
+                        hW[i].copy_(Ws[i], non_blocking=True)
+                    if g == 0 and tail_n:
+                        htp.copy_(tp, non_blocking=True)
+            stream.wait_stream(s_out)                # the step ends when the last parameter is on the host
 
         for _ in range(max(1, min(args.warmup, 3))):
             e2e_step()
@@ -332,9 +370,13 @@ def run_ours(args) -> int:
             dist.barrier()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / k_e2e)
         e2e = {"value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": k_e2e,
-               "what": "per step: pinned H2D of every gradient (and tail grad), the step through the C ABI, "
-                       "D2H of every updated parameter (and tail param); optimizer state resident"}
+               "d2h_bytes_per_step": int(d2h), "steps": k_e2e, "groups": len(groups),
+               "what": "per step: pinned H2D of every gradient (and the tail grad), the step through the C ABI "
+                       f"in {len(groups)} groups whose copies overlap each other's compute, D2H of every "
+                       "updated parameter (and the tail param); optimizer state resident"}
+        for st_ in gsteps:
+            st_.close()
+        del gsteps
 
     # 64 Mi-element tail (the skew workload's tail size): AdamW GB/s alone
     tail_bench = None
@@ -502,6 +544,7 @@ def main(argv=None) -> int:
     ap.add_argument("--mode", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-groups", type=int, default=4, help="matrix groups pipelined in the e2e measurement")
     ap.add_argument("--no-tail-bench", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")

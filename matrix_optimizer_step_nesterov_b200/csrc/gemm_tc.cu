@@ -11,9 +11,9 @@
 // 4-stage TMA ring; a double-buffered 2 x 256-column fp32 accumulator in TMEM
 // lets the epilogue of one tile overlap the mainloop of the next.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues the MMAs (one elected lane), warps 2-5 run the epilogue, one TMEM
-// lane quadrant (32 rows) each.  Every mbarrier wait is bounded: past the
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues the MMAs (one elected lane), warps 2-9 run the epilogue, two per TMEM
+// lane quadrant (32 rows), each on half of the tile's columns.  Every mbarrier wait is bounded: past the
 // limit the waiting thread records MFSDP_ERR_TIMEOUT in the device status
 // word, raises a CTA-wide abort flag and returns; the other roles see the flag
 // in their own waits, the producer drains the loads it has in flight, and
@@ -39,8 +39,10 @@ constexpr int A_BYTES = BM * BK * 2;            // 16 KiB
 constexpr int B_BYTES = BN * BK * 2;            // 32 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KiB
 constexpr int TMEM_COLS = 2 * BN;               // two fp32 accumulators
-constexpr int NUM_THREADS = 192;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+constexpr int NUM_EPI_WARPS = 8;                // two per TMEM lane quadrant, each half the columns
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int STG_BYTES = NUM_EPI_WARPS * 32 * 33 * 4;   // epilogue staging: one 32 x 33 fp32 buffer per epilogue warp
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 // per-matrix TMA descriptors, stored in the workspace head (64-byte aligned)
@@ -175,91 +177,199 @@ __host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major) {
 __device__ __forceinline__ void store_bf16(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
 // ---------------------------------------------------------------------------
-// epilogue of one 32-column chunk held by one thread (row gi, columns gj0 + t)
+// Warp-cooperative epilogue of one 32 x 32 chunk of the accumulator.
+// TMEM delivers it in the row domain: lane l holds row gi0 + l, columns
+// gj0 .. gj0 + 31.  Accesses that run along a column (the mirrored triangle
+// of a symmetric result, the transposed parameter write) are issued straight
+// from the row domain, where the 32 lanes touch 32 consecutive elements.
+// Accesses that run along a row go through the warp's 32 x 33 staging buffer
+// into the column domain (lane l takes column gj0 + l, rows one by one), so
+// they are coalesced too.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void epilogue_chunk(int ph, const MatDev& md, int iter, const StepScalars& sc,
-                                               float sg, int gi, int gj0, int Ncols, const uint32_t (&r)[32]) {
-    const int cur = iter & 1, nxt = cur ^ 1;
-    if (ph == PH_GRAM) {
+template <int ph>
+__device__ __forceinline__ void epilogue_chunk_warp(const MatDev& md, int iter, const StepScalars& sc,
+                                                    float sg, int gi0, int gj0, int Mrows, int Ncols,
+                                                    const uint32_t (&r)[32], float (*stg)[33], int lane) {
+    const int nxt = (iter & 1) ^ 1;
+    const int gi = gi0 + lane;      // row domain: this lane's row
+    const int gjc = gj0 + lane;     // column domain: this lane's column
+    const bool row_ok = gi < Mrows;
+    const bool col_ok = gjc < Ncols;
+    const int64_t lda = md.lda;
+    // Every global load of a chunk is issued before any result is used, so the
+    // 32 loads of a lane are in flight together.
+    if (ph == PH_GRAM || ph == PH_POLY) {
+        // symmetric result: each element with row <= col is stored to both triangles
+        __nv_bfloat16* ob = (ph == PH_GRAM) ? md.ab : static_cast<__nv_bfloat16*>(md.bm);
+        float ev[32];
+        float di = 0.f, dj = 0.f;
+        if (ph == PH_POLY) {
+            // E_A is symmetric: E[gi][gj] is read as E[gj][gi], consecutive across lanes
+            #pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const int gj = gj0 + t;
+                ev[t] = (row_ok && gj < Ncols && gi < gj) ? md.af[(int64_t)gj * lda + gi] : 0.f;
+            }
+            di = row_ok ? md.da[gi] : 0.f;
+            dj = col_ok ? md.da[gjc] : 0.f;
+        }
         const float s2 = sg * sg;
         #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const int gj = gj0 + t;
-            if (gj >= Ncols || gi > gj) continue;
-            const float v = s2 * __uint_as_float(r[t]);
-            if (gi == gj) {
-                md.da[gi] = v;
-                md.af[(int64_t)gi * md.lda + gi] = 0.f;
-                store_bf16(md.ab + (int64_t)gi * md.lda + gi, 0.f);
-            } else {
-                md.af[(int64_t)gi * md.lda + gj] = v;
-                md.af[(int64_t)gj * md.lda + gi] = v;
-                store_bf16(md.ab + (int64_t)gi * md.lda + gj, v);
-                store_bf16(md.ab + (int64_t)gj * md.lda + gi, v);
-            }
-        }
-    } else if (ph == PH_POLY) {
-        __nv_bfloat16* bm = static_cast<__nv_bfloat16*>(md.bm);
-        const float di = md.da[gi];
-        #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int gj = gj0 + t;
-            if (gj >= Ncols || gi > gj) continue;
             const float acc = __uint_as_float(r[t]);
-            if (gi == gj) {
-                md.db[gi] = sc.b * di + sc.c * fmaf(di, di, acc);
-                store_bf16(bm + (int64_t)gi * md.lda + gi, 0.f);
-            } else {
-                const float e = md.af[(int64_t)gi * md.lda + gj];
-                const float v = sc.b * e + sc.c * fmaf(di + md.da[gj], e, acc);
-                store_bf16(bm + (int64_t)gi * md.lda + gj, v);
-                store_bf16(bm + (int64_t)gj * md.lda + gi, v);
+            const float dt = (ph == PH_POLY) ? __shfl_sync(0xffffffffu, dj, t) : 0.f;   // d_A of column gj
+            float val = 0.f;
+            if (row_ok && gj < Ncols && gi <= gj) {
+                if (ph == PH_GRAM) {
+                    val = s2 * acc;
+                    if (gi == gj) {
+                        md.da[gi] = val;
+                        md.af[(int64_t)gi * lda + gi] = 0.f;
+                        ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
+                    } else {
+                        md.af[(int64_t)gj * lda + gi] = val;          // lower triangle, along column gj
+                        ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
+                    }
+                } else {
+                    if (gi == gj) {
+                        md.db[gi] = sc.b * di + sc.c * fmaf(di, di, acc);
+                        ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
+                    } else {
+                        const float e = ev[t];
+                        val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
+                        ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
+                    }
+                }
+            }
+            stg[lane][t] = val;
+        }
+        __syncwarp();
+        // column domain: the upper-triangle copies (row gi0 + rr < column gjc)
+        #pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            const int gi2 = gi0 + rr;
+            if (gi2 < Mrows && col_ok && gi2 < gjc) {
+                const float val = stg[rr][lane];
+                if (ph == PH_GRAM) md.af[(int64_t)gi2 * lda + gjc] = val;
+                ob[(int64_t)gi2 * lda + gjc] = __float2bfloat16_rn(val);
             }
         }
-    } else {
-        const float f = sc.a + md.db[gi];
-        float* xrow = md.xf[0] + (int64_t)gi * md.ldx;
-        if (ph == PH_APPLY) {
-            __nv_bfloat16* xbn = md.xb[nxt] + (int64_t)gi * md.ldx;
+        __syncwarp();
+        return;
+    }
+    // APPLY / FINAL: X_new = s ((a + d_B,i) X + E_B X), computed in the column domain
+    float* xf = md.xf[0];
+    const int64_t ldx = md.ldx;
+    #pragma unroll
+    for (int t = 0; t < 32; ++t) stg[lane][t] = __uint_as_float(r[t]);
+    const float fa = row_ok ? (sc.a + md.db[gi]) : 0.f;
+    __syncwarp();
+    if (ph == PH_APPLY) {
+        __nv_bfloat16* xbn = md.xb[nxt];
+        const float* xcol = xf + (int64_t)gi0 * ldx + gjc;
+        #pragma unroll 1
+        for (int h = 0; h < 32; h += 16) {          // 16 loads in flight per lane
+            float xv[16];
             #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const int gj = gj0 + t;
-                if (gj >= Ncols) continue;
-                const float v = sg * fmaf(f, xrow[gj], __uint_as_float(r[t]));
-                xrow[gj] = v;
-                store_bf16(xbn + gj, v);
-            }
-        } else {
+            for (int k = 0; k < 16; ++k)
+                xv[k] = (gi0 + h + k < Mrows && col_ok) ? xcol[(int64_t)(h + k) * ldx] : 0.f;
             #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const int gj = gj0 + t;
-                if (gj >= Ncols) continue;
-                const float o = md.shape_scale * (sg * fmaf(f, xrow[gj], __uint_as_float(r[t])));
-                const int64_t widx = md.tr ? (int64_t)gj * md.cols + gi : (int64_t)gi * md.cols + gj;
-                if (md.update_out) md.update_out[widx] = o;
-                if (md.param_bf16) {
-                    __nv_bfloat16* w = static_cast<__nv_bfloat16*>(md.param);
-                    w[widx] = __float2bfloat16_rn(fmaf(-sc.lr, o, __bfloat162float(w[widx]) * sc.decay));
-                } else {
-                    float* w = static_cast<float*>(md.param);
-                    w[widx] = fmaf(-sc.lr, o, w[widx] * sc.decay);
+            for (int k = 0; k < 16; ++k) {
+                const int rr = h + k;
+                const float f = __shfl_sync(0xffffffffu, fa, rr);
+                if (gi0 + rr < Mrows && col_ok) {
+                    const int64_t idx = (int64_t)(gi0 + rr) * ldx + gjc;
+                    const float v = sg * fmaf(f, xv[k], stg[rr][lane]);
+                    xf[idx] = v;
+                    xbn[idx] = __float2bfloat16_rn(v);
                 }
             }
         }
+        __syncwarp();
+        return;
     }
+    float xv[32];
+    #pragma unroll
+    for (int rr = 0; rr < 32; ++rr) {
+        const int gi2 = gi0 + rr;
+        xv[rr] = (gi2 < Mrows && col_ok) ? xf[(int64_t)gi2 * ldx + gjc] : 0.f;
+    }
+    // FINAL: O = scale * X_new, W <- W (1 - lr wd) - lr O, at W[i][j] or, transposed, W[j][i]
+    const int64_t cols = md.cols;
+    #pragma unroll
+    for (int rr = 0; rr < 32; ++rr) {
+        const float f = __shfl_sync(0xffffffffu, fa, rr);
+        xv[rr] = md.shape_scale * (sg * fmaf(f, xv[rr], stg[rr][lane]));   // O, column domain
+    }
+    if (!md.tr) {
+        float wv[32];
+        #pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            const int gi2 = gi0 + rr;
+            const int64_t widx = (int64_t)gi2 * cols + gjc;
+            wv[rr] = 0.f;
+            if (gi2 < Mrows && col_ok)
+                wv[rr] = md.param_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(md.param)[widx])
+                                       : static_cast<const float*>(md.param)[widx];
+        }
+        #pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            const int gi2 = gi0 + rr;
+            if (gi2 < Mrows && col_ok) {
+                const int64_t widx = (int64_t)gi2 * cols + gjc;
+                const float o = xv[rr];
+                if (md.update_out) md.update_out[widx] = o;
+                const float w = fmaf(-sc.lr, o, wv[rr] * sc.decay);
+                if (md.param_bf16) static_cast<__nv_bfloat16*>(md.param)[widx] = __float2bfloat16_rn(w);
+                else static_cast<float*>(md.param)[widx] = w;
+            }
+        }
+        __syncwarp();
+        return;
+    }
+    // transposed parameter: back to the row domain, W[j][i] consecutive across lanes
+    #pragma unroll
+    for (int rr = 0; rr < 32; ++rr) stg[rr][lane] = xv[rr];
+    __syncwarp();
+    float wv[32];
+    #pragma unroll
+    for (int t = 0; t < 32; ++t) {
+        const int gj = gj0 + t;
+        const int64_t widx = (int64_t)gj * cols + gi;
+        wv[t] = 0.f;
+        if (row_ok && gj < Ncols)
+            wv[t] = md.param_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(md.param)[widx])
+                                  : static_cast<const float*>(md.param)[widx];
+    }
+    #pragma unroll
+    for (int t = 0; t < 32; ++t) {
+        const int gj = gj0 + t;
+        if (row_ok && gj < Ncols) {
+            const int64_t widx = (int64_t)gj * cols + gi;
+            const float o = stg[lane][t];
+            if (md.update_out) md.update_out[widx] = o;
+            const float w = fmaf(-sc.lr, o, wv[t] * sc.decay);
+            if (md.param_bf16) static_cast<__nv_bfloat16*>(md.param)[widx] = __float2bfloat16_rn(w);
+            else static_cast<float*>(md.param)[widx] = w;
+        }
+    }
+    __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
 // the persistent kernel
 // ---------------------------------------------------------------------------
+template <int ph>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps, int32_t nmats,
+tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps, int32_t nmats,
                 const TileDev* __restrict__ tiles, int32_t ntiles, int32_t iter, StepScalars sc,
                 const float* __restrict__ s, int32_t* status) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned stage ring (128 B swizzle atoms need 1024 B alignment)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    float* stg_all = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + STG_BYTES);
     // bars: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], mma_done
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -276,7 +386,7 @@ tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __res
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(tfull0 + 8 * i, 1);
-            mbar_init(tempty0 + 8 * i, 4);   // one arrive per epilogue warp
+            mbar_init(tempty0 + 8 * i, NUM_EPI_WARPS);   // one arrive per epilogue warp
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -386,8 +496,9 @@ tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __res
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 2..9) ----------------
         const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+        const int half = (warp - 2) >> 2;          // which 128 of the tile's 256 columns
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -401,15 +512,19 @@ tc_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, const TcMaps* __res
             if (!ok) break;
             tc_fence_after();
             const float sg = (iter == 0) ? s[td.mat] : 1.0f;
-            const int gi = td.tm * BM + quad * 32 + lane;
+            const int gi0 = td.tm * BM + quad * 32;
             const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
-            // skip whole chunks that lie left of the diagonal in symmetric phases
+            float (*stg)[33] = reinterpret_cast<float (*)[33]>(stg_all + (warp - 2) * 32 * 33);
             #pragma unroll 1
-            for (int q = 0; q < BN / 32; ++q) {
+            for (int q = half * (BN / 64); q < (half + 1) * (BN / 64); ++q) {
                 const int gj0 = td.tn * BN + q * 32;
+                // warp-uniform skips: rows or columns out of range, or (symmetric
+                // phases) a chunk entirely below the diagonal
+                if (gi0 >= Mrows || gj0 >= Ncols) continue;
+                if (!gemm && gj0 + 31 < gi0) continue;
                 uint32_t r[32];
-                tmem_ld32(trow + q * 32, r);       // warp-collective: every lane executes it
-                if (gi < Mrows && gj0 < Ncols) epilogue_chunk(ph, md, iter, sc, sg, gi, gj0, Ncols, r);
+                tmem_ld32(trow + q * 32, r);       // warp-collective
+                epilogue_chunk_warp<ph>(md, iter, sc, sg, gi0, gj0, Mrows, Ncols, r, stg, lane);
             }
             tc_fence_before();
             __syncwarp();
@@ -515,7 +630,10 @@ cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, i
     static int sms = 0;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc_phase_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(tc_phase_kernel<PH_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_phase_kernel<PH_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_phase_kernel<PH_APPLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_phase_kernel<PH_FINAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         int dev = 0;
         cudaGetDevice(&dev);
@@ -524,8 +642,22 @@ cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, i
         attr_set = true;
     }
     const int grid = std::min(ntiles, sms);
-    tc_phase_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ph, d_mats, static_cast<const TcMaps*>(d_maps), nmats,
-                                                           d_tiles, ntiles, iter, sc, s, device_status_ptr());
+    const TcMaps* maps = static_cast<const TcMaps*>(d_maps);
+    int32_t* status = device_status_ptr();
+    switch (ph) {
+        case PH_GRAM:
+            tc_phase_kernel<PH_GRAM><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, status);
+            break;
+        case PH_POLY:
+            tc_phase_kernel<PH_POLY><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, status);
+            break;
+        case PH_APPLY:
+            tc_phase_kernel<PH_APPLY><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, status);
+            break;
+        default:
+            tc_phase_kernel<PH_FINAL><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, status);
+            break;
+    }
     return cudaGetLastError();
 }
 
