@@ -89,6 +89,18 @@ def split_groups(specs, n_groups: int) -> List[List[int]]:
     return [grp for grp in groups if grp]
 
 
+def bench_workload(args):
+    """The named workload, or a single-owner list of explicit shapes (--shapes RxC,RxC)."""
+    from synth import workload
+    from synth.workloads import custom_workload
+    if args.shapes:
+        shapes = [tuple(int(v) for v in sh.lower().split("x")) for sh in args.shapes.split(",")]
+        dtype = "bf16" if args.mode == "bf16" else "f32"
+        return custom_workload(shapes, dtype=dtype, tail=args.tail, seed=4242, spike_rule="rank:4:rel:10",
+                               name="shapes " + args.shapes)
+    return workload(args.workload)
+
+
 def max_over_ranks(x: float) -> float:
     import torch
     import torch.distributed as dist
@@ -248,7 +260,7 @@ def run_ours(args) -> int:
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
 
-    wl = workload(args.workload)
+    wl = bench_workload(args)
     R = wl.world_size or 1
     if wl.world_size is None:
         specs, owns_tail, planned = wl.matrices, True, 0
@@ -507,7 +519,7 @@ def run_reference(args) -> int:
         return 0
     from synth import workload
     import oracle
-    wl = workload(args.workload)
+    wl = bench_workload(args)
     R = wl.world_size or 1
     if wl.world_size is None:
         specs, owns_tail = wl.matrices, True
@@ -542,6 +554,8 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="7b_share")
     ap.add_argument("--mode", default="bf16", choices=["bf16", "fp32"])
+    ap.add_argument("--shapes", default="", help="explicit matrix list RxC,RxC (profiling cases) instead of --workload")
+    ap.add_argument("--tail", type=int, default=0, help="tail length with --shapes")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-groups", type=int, default=4, help="matrix groups pipelined in the e2e measurement")

@@ -31,19 +31,29 @@
 namespace mfsdp {
 namespace {
 
-constexpr int BM = 128;          // tile rows (MMA M)
+constexpr int BM = 128;          // rows of the output tile held by one CTA (TMEM lanes)
 constexpr int BN = 256;          // tile cols (MMA N)
 constexpr int BK = 64;           // K per stage: one 128 B swizzle atom of bf16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;            // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;            // 32 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KiB
+constexpr int A_BYTES = BM * BK * 2;            // 16 KiB per CTA per stage
 constexpr int TMEM_COLS = 2 * BN;               // two fp32 accumulators
 constexpr int NUM_EPI_WARPS = 8;                // two per TMEM lane quadrant, each half the columns
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int STG_BYTES = NUM_EPI_WARPS * 32 * 33 * 4;   // epilogue staging: one 32 x 33 fp32 buffer per epilogue warp
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+// CTAs per MMA: 1 (cta_group::1, M = 128) or 2 (a cluster pair running
+// cta_group::2 MMAs of M = 256; each CTA loads its own 128 rows of A and half
+// of B, the MMA reads B across the pair, so each SM fetches 32 KiB instead
+// of 48 KiB per 64-deep K block).
+template <int CG>
+struct TcCfg {
+    static constexpr int B_ROWS = BN / CG;                      // B rows (N) this CTA loads
+    static constexpr int STAGE_BYTES = A_BYTES + B_ROWS * BK * 2;
+    static constexpr int STAGES = CG == 1 ? 4 : 6;
+    static constexpr int TILE_M = BM * CG;                      // rows of a tile
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+};
+constexpr int kCtaGroup = 2;      // the engine's configuration
 
 // per-matrix TMA descriptors, stored in the workspace head (64-byte aligned)
 struct alignas(64) TcMaps {
@@ -116,6 +126,59 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA load of this CTA's share of a cta_group::2 operand; completion is
+// counted on the barrier at `bar_cluster` (the leader CTA's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_mma2(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// arrive on the barrier at this offset in both CTAs of the pair once the
+// issuing thread's prior cta_group::2 MMAs complete
+__device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(bar), "h"((uint16_t)0x3) : "memory");
+}
+
+__device__ __forceinline__ void tc_commit2_local(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -164,17 +227,15 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
     return d;
 }
 
-// Instruction descriptor: D fp32, A/B bf16, A K-major, B K- or MN-major, N=256, M=128.
-__host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major) {
+// Instruction descriptor: D fp32, A/B bf16, A K-major, B K- or MN-major, N = 256, M = 128 or 256.
+__host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major, int m) {
     return (1u << 4)                 // D format: F32
          | (1u << 7)                 // A format: BF16
          | (1u << 10)                // B format: BF16
          | ((b_mn_major ? 1u : 0u) << 16)
          | (static_cast<uint32_t>(BN >> 3) << 17)
-         | (static_cast<uint32_t>(BM >> 4) << 24);
+         | (static_cast<uint32_t>(m >> 4) << 24);
 }
-
-__device__ __forceinline__ void store_bf16(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
 // ---------------------------------------------------------------------------
 // Warp-cooperative epilogue of one 32 x 32 chunk of the accumulator.
@@ -357,14 +418,80 @@ __device__ __forceinline__ void epilogue_chunk_warp(const MatDev& md, int iter, 
     __syncwarp();
 }
 
+// APPLY epilogue of one warp over its chunks [qa, qb) of a tile, software
+// pipelined: the 16 master-X loads of the next half-chunk are issued before
+// the current half-chunk is computed and stored, so global latency overlaps
+// the stores and the TMEM reads.
+__device__ __forceinline__ void epilogue_apply_warp(const MatDev& md, int iter, const StepScalars& sc, float sg,
+                                                    int gi0, int gj_tile, int qa, int qb, int Mrows, int Ncols,
+                                                    uint32_t trow, float (*stg)[33], int lane) {
+    const int nxt = (iter & 1) ^ 1;
+    float* xf = md.xf[0];
+    __nv_bfloat16* xbn = md.xb[nxt];
+    const int64_t ldx = md.ldx;
+    const int gi = gi0 + lane;
+    const float fa = gi < Mrows ? (sc.a + md.db[gi]) : 0.f;
+    // chunks [qa, qe) hold at least one column in range (rows checked by the caller)
+    int qe = qa;
+    while (qe < qb && gj_tile + qe * 32 < Ncols) ++qe;
+    const int nb = 2 * (qe - qa);                 // half-chunks of 16 rows
+    if (nb == 0) return;
+    auto load_half = [&](int b, float (&xv)[16]) {
+        const int gjc = gj_tile + (qa + (b >> 1)) * 32 + lane;
+        const int h = (b & 1) * 16;
+        const bool ok = gjc < Ncols;
+        const float* p = xf + (int64_t)(gi0 + h) * ldx + gjc;
+        #pragma unroll
+        for (int k = 0; k < 16; ++k) xv[k] = (ok && gi0 + h + k < Mrows) ? p[(int64_t)k * ldx] : 0.f;
+    };
+    float cur[16], nx[16];
+    load_half(0, cur);
+    #pragma unroll 1
+    for (int b = 0; b < nb; ++b) {
+        const int q = qa + (b >> 1);
+        const int h = (b & 1) * 16;
+        if (h == 0) {
+            uint32_t r[32];
+            tmem_ld32(trow + q * 32, r);          // warp-collective
+            __syncwarp();                         // previous chunk's reads of stg are done
+            #pragma unroll
+            for (int t = 0; t < 32; ++t) stg[lane][t] = __uint_as_float(r[t]);
+            __syncwarp();
+        }
+        if (b + 1 < nb) load_half(b + 1, nx);
+        float fk[16];                             // (a + d_B) of the 16 rows, gathered by every lane
+        #pragma unroll
+        for (int k = 0; k < 16; ++k) fk[k] = __shfl_sync(0xffffffffu, fa, h + k);
+        const int gjc = gj_tile + q * 32 + lane;
+        if (gjc < Ncols) {
+            #pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int rr = h + k;
+                if (gi0 + rr < Mrows) {
+                    const int64_t idx = (int64_t)(gi0 + rr) * ldx + gjc;
+                    const float v = sg * fmaf(fk[k], cur[k], stg[rr][lane]);
+                    xf[idx] = v;
+                    xbn[idx] = __float2bfloat16_rn(v);
+                }
+            }
+        }
+        #pragma unroll
+        for (int k = 0; k < 16; ++k) cur[k] = nx[k];
+    }
+    __syncwarp();
+}
+
 // ---------------------------------------------------------------------------
 // the persistent kernel
 // ---------------------------------------------------------------------------
-template <int ph>
+template <int ph, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps, int32_t nmats,
                 const TileDev* __restrict__ tiles, int32_t ntiles, int32_t iter, StepScalars sc,
                 const float* __restrict__ s, int32_t* status) {
+    using C = TcCfg<CG>;
+    constexpr int STAGES = C::STAGES;
+    constexpr int STAGE_BYTES = C::STAGE_BYTES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned stage ring (128 B swizzle atoms need 1024 B alignment)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -378,6 +505,9 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
     const uint32_t tfull0 = smem_u32(bars + 2 * STAGES), tempty0 = smem_u32(bars + 2 * STAGES + 2);
     const uint32_t mma_done = smem_u32(bars + 2 * STAGES + 4);
+    const uint32_t rank = (CG == 2) ? cluster_rank() : 0u;      // 0 = leader (issues the MMAs)
+    const bool leader = rank == 0;
+    const int cluster_id = blockIdx.x / CG, nclusters = gridDim.x / CG;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -386,27 +516,34 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(tfull0 + 8 * i, 1);
-            mbar_init(tempty0 + 8 * i, NUM_EPI_WARPS);   // one arrive per epilogue warp
+            mbar_init(tempty0 + 8 * i, CG * NUM_EPI_WARPS);   // one arrive per epilogue warp of the pair
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if (CG == 2) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync();     // the peer's barriers are initialised before anyone signals them
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const bool gemm = (ph == PH_APPLY || ph == PH_FINAL);
+    constexpr bool gemm = (ph == PH_APPLY || ph == PH_FINAL);
     const int cur = iter & 1;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producer (both CTAs) ----------------
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
@@ -414,7 +551,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             int issued[STAGES];                  // parity of the last fill issued per stage, -1 = none
             #pragma unroll
             for (int i = 0; i < STAGES; ++i) issued[i] = -1;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int t = cluster_id; t < ntiles && ok; t += nclusters) {
                 const TileDev td = tiles[t];
                 const MatDev& md = mats[td.mat];
                 const TcMaps& mp = maps[td.mat];
@@ -422,27 +559,44 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                 const int nk = (K + BK - 1) / BK;
                 const CUtensorMap* amap = (ph == PH_GRAM) ? &mp.xk[cur] : (ph == PH_POLY) ? &mp.ea : &mp.eb;
                 const CUtensorMap* bmap = (ph == PH_GRAM) ? &mp.xk[cur] : (ph == PH_POLY) ? &mp.ea : &mp.xm[cur];
-                const int i0 = td.tm * BM, j0 = td.tn * BN;
+                const int i0 = td.tm * C::TILE_M + (int)rank * BM;        // this CTA's A rows
+                const int jb = td.tn * BN + (int)rank * C::B_ROWS;        // this CTA's share of B
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!wait_bounded(empty0 + 8 * stage, phase ^ 1, abort_flag, status)) { ok = false; break; }
                     const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
                     const uint32_t sb = sa + A_BYTES;
                     const uint32_t fb = full0 + 8 * stage;
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                    tma_load_2d(sa, amap, fb, kb * BK, i0);
-                    if (!gemm) {
-                        tma_load_2d(sb, bmap, fb, kb * BK, j0);
-                        tma_load_2d(sb + BN / 2 * BK * 2, bmap, fb, kb * BK, j0 + BN / 2);
+                    if (CG == 1) {
+                        mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                        tma_load_2d(sa, amap, fb, kb * BK, i0);
+                        if (!gemm) {
+                            #pragma unroll
+                            for (int h = 0; h < C::B_ROWS / 128; ++h)
+                                tma_load_2d(sb + h * (128 * BK * 2), bmap, fb, kb * BK, jb + 128 * h);
+                        } else {
+                            #pragma unroll
+                            for (int q = 0; q < C::B_ROWS / 64; ++q)
+                                tma_load_2d(sb + q * (BK * 128), bmap, fb, jb + 64 * q, kb * BK);
+                        }
                     } else {
-                        #pragma unroll
-                        for (int q = 0; q < BN / 64; ++q)
-                            tma_load_2d(sb + q * (BK * 128), bmap, fb, j0 + 64 * q, kb * BK);
+                        if (leader) mbar_arrive_expect_tx(fb, CG * STAGE_BYTES);   // both CTAs' bytes
+                        const uint32_t fbl = map_to_rank(fb, 0);
+                        tma_load_2d_pair(sa, amap, fbl, kb * BK, i0);
+                        if (!gemm) {
+                            #pragma unroll
+                            for (int h = 0; h < C::B_ROWS / 128; ++h)
+                                tma_load_2d_pair(sb + h * (128 * BK * 2), bmap, fbl, kb * BK, jb + 128 * h);
+                        } else {
+                            #pragma unroll
+                            for (int q = 0; q < C::B_ROWS / 64; ++q)
+                                tma_load_2d_pair(sb + q * (BK * 128), bmap, fbl, jb + 64 * q, kb * BK);
+                        }
                     }
                     issued[stage] = static_cast<int>(phase);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
-            if (!ok) {
+            if (!ok && leader) {
                 // aborting: wait (bounded, 10 ms each) until every issued load has landed
                 for (int i = 0; i < STAGES; ++i) {
                     if (issued[i] < 0) continue;
@@ -454,15 +608,15 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc(gemm);
+        // ---------------- MMA issuer (leader CTA) ----------------
+        if (lane == 0 && leader) {
+            const uint32_t idesc = make_idesc(gemm, C::TILE_M);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int t = cluster_id; t < ntiles && ok; t += nclusters) {
                 const TileDev td = tiles[t];
                 const MatDev& md = mats[td.mat];
                 const int K = (ph == PH_GRAM) ? md.c : md.r;
@@ -480,28 +634,35 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                         const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024);
                         const uint64_t bd = gemm ? smem_desc(sb + kk * 16 * 128, BK * 128, 1024)
                                                  : smem_desc(sb + kk * 32, 16, 1024);
-                        tc_mma(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        if (CG == 2) tc_mma2(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        else tc_mma(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
-                    tc_commit(empty0 + 8 * stage);     // stage free once these MMAs finish
+                    // stage free (in both CTAs) once these MMAs finish
+                    if (CG == 2) tc_commit2_both(empty0 + 8 * stage);
+                    else tc_commit(empty0 + 8 * stage);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                tc_commit(tfull0 + 8 * acc);           // accumulator ready for the epilogue
+                // accumulator ready for the epilogue (of both CTAs)
+                if (CG == 2) tc_commit2_both(tfull0 + 8 * acc);
+                else tc_commit(tfull0 + 8 * acc);
                 if (++acc == 2) { acc = 0; acc_phase ^= 1; }
             }
             // every MMA this thread issued has completed before TMEM is freed (bounded)
-            tc_commit(mma_done);
+            if (CG == 2) tc_commit2_local(mma_done);
+            else tc_commit(mma_done);
             const unsigned long long t0 = globaltimer();
             while (!mbar_try_wait(mma_done, 0) && globaltimer() - t0 < 100000000ull) {
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..9) ----------------
+        // ---------------- epilogue (warps 2..9, both CTAs) ----------------
         const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
         const int half = (warp - 2) >> 2;          // which 128 of the tile's 256 columns
+        const uint32_t tempty_leader0 = (CG == 2) ? map_to_rank(tempty0, 0) : tempty0;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        for (int t = cluster_id; t < ntiles; t += nclusters) {
             const TileDev td = tiles[t];
             const MatDev& md = mats[td.mat];
             const int Mrows = md.r;
@@ -512,33 +673,47 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             if (!ok) break;
             tc_fence_after();
             const float sg = (iter == 0) ? s[td.mat] : 1.0f;
-            const int gi0 = td.tm * BM + quad * 32;
+            const int gi0 = td.tm * C::TILE_M + (int)rank * BM + quad * 32;
             const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
             float (*stg)[33] = reinterpret_cast<float (*)[33]>(stg_all + (warp - 2) * 32 * 33);
-            #pragma unroll 1
-            for (int q = half * (BN / 64); q < (half + 1) * (BN / 64); ++q) {
-                const int gj0 = td.tn * BN + q * 32;
-                // warp-uniform skips: rows or columns out of range, or (symmetric
-                // phases) a chunk entirely below the diagonal
-                if (gi0 >= Mrows || gj0 >= Ncols) continue;
-                if (!gemm && gj0 + 31 < gi0) continue;
-                uint32_t r[32];
-                tmem_ld32(trow + q * 32, r);       // warp-collective
-                epilogue_chunk_warp<ph>(md, iter, sc, sg, gi0, gj0, Mrows, Ncols, r, stg, lane);
+            if constexpr (ph == PH_APPLY) {
+                if (gi0 < Mrows)
+                    epilogue_apply_warp(md, iter, sc, sg, gi0, td.tn * BN, half * (BN / 64), (half + 1) * (BN / 64),
+                                        Mrows, Ncols, trow, stg, lane);
+            } else {
+                #pragma unroll 1
+                for (int q = half * (BN / 64); q < (half + 1) * (BN / 64); ++q) {
+                    const int gj0 = td.tn * BN + q * 32;
+                    // warp-uniform skips: rows or columns out of range, or (symmetric
+                    // phases) a chunk entirely below the diagonal
+                    if (gi0 >= Mrows || gj0 >= Ncols) continue;
+                    if (!gemm && gj0 + 31 < gi0) continue;
+                    uint32_t r[32];
+                    tmem_ld32(trow + q * 32, r);       // warp-collective
+                    epilogue_chunk_warp<ph>(md, iter, sc, sg, gi0, gj0, Mrows, Ncols, r, stg, lane);
+                }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+            if (lane == 0) {
+                if (CG == 2) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
+                else mbar_arrive(tempty0 + 8 * acc);
+            }
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync();     // neither CTA frees TMEM or exits while its peer may still use it
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
-                     : "memory");
+        if (CG == 2)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                         : "memory");
     }
 }
 
@@ -596,15 +771,16 @@ bool tc_encode_maps(const std::vector<MatDev>& mats, void* host_out) {
 
 void tc_build_tiles(const std::vector<MatDev>& mats, std::vector<TileDev>& gram, std::vector<TileDev>& poly,
                     std::vector<TileDev>& gen) {
+    constexpr int TM = TcCfg<kCtaGroup>::TILE_M;
     for (int32_t mi = 0; mi < static_cast<int32_t>(mats.size()); ++mi) {
         const MatDev& m = mats[mi];
-        const int tm_n = (m.r + BM - 1) / BM;
+        const int tm_n = (m.r + TM - 1) / TM;
         const int tn_sym = (m.r + BN - 1) / BN;
         const int tn_gen = (m.c + BN - 1) / BN;
         for (int i = 0; i < tm_n; ++i) {
             for (int j = 0; j < tn_sym; ++j) {
-                // keep tiles that reach the upper triangle (row i*BM <= last column of the tile)
-                if (i * BM > j * BN + BN - 1) continue;
+                // keep tiles that reach the upper triangle (first row <= last column of the tile)
+                if (i * TM > j * BN + BN - 1) continue;
                 gram.push_back({mi, i, j, (m.c + BK - 1) / BK});
                 poly.push_back({mi, i, j, (m.r + BK - 1) / BK});
             }
@@ -618,46 +794,82 @@ void tc_build_tiles(const std::vector<MatDev>& mats, std::vector<TileDev>& gram,
         if (a.tm != b.tm) return a.tm < b.tm;
         return a.tn < b.tn;
     };
+    // APPLY: column blocks outer, so that a wave of CTAs shares one slice of X
+    // and the whole (small) E_B instead of streaming all of X per wave
+    auto lpt_cols = [](const TileDev& a, const TileDev& b) {
+        if (a.kblk != b.kblk) return a.kblk > b.kblk;
+        if (a.mat != b.mat) return a.mat < b.mat;
+        if (a.tn != b.tn) return a.tn < b.tn;
+        return a.tm < b.tm;
+    };
     std::stable_sort(gram.begin(), gram.end(), lpt);
     std::stable_sort(poly.begin(), poly.end(), lpt);
-    std::stable_sort(gen.begin(), gen.end(), lpt);
+    std::stable_sort(gen.begin(), gen.end(), lpt_cols);
 }
+
+namespace {
+
+template <int ph>
+cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats, const TileDev* d_tiles,
+                         int32_t ntiles, int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st,
+                         int sms) {
+    constexpr int CG = kCtaGroup;
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(tc_phase_kernel<ph, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   TcCfg<CG>::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    static int max_clusters = 0;      // clusters of CG CTAs that fit on the device at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((sms / CG) * CG, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = TcCfg<CG>::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_clusters == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, tc_phase_kernel<ph, CG>, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = sms / CG;
+        }
+        max_clusters = n;
+    }
+    const int clusters = std::max(1, std::min(ntiles, max_clusters));
+    cfg.gridDim = dim3(clusters * CG, 1, 1);
+    return cudaLaunchKernelEx(&cfg, tc_phase_kernel<ph, CG>, d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s,
+                              device_status_ptr());
+}
+
+}  // namespace
 
 cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, int32_t nmats,
                            const TileDev* d_tiles, int32_t ntiles, int32_t iter, const StepScalars& sc,
                            const float* s, cudaStream_t st) {
     if (ntiles <= 0) return cudaSuccess;
     static int sms = 0;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc_phase_kernel<PH_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_phase_kernel<PH_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_phase_kernel<PH_APPLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(tc_phase_kernel<PH_FINAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
+    if (sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (sms <= 0) sms = 148;
-        attr_set = true;
     }
-    const int grid = std::min(ntiles, sms);
     const TcMaps* maps = static_cast<const TcMaps*>(d_maps);
-    int32_t* status = device_status_ptr();
+    cudaError_t e;
     switch (ph) {
-        case PH_GRAM:
-            tc_phase_kernel<PH_GRAM><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, status);
-            break;
-        case PH_POLY:
-            tc_phase_kernel<PH_POLY><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, status);
-            break;
-        case PH_APPLY:
-            tc_phase_kernel<PH_APPLY><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, status);
-            break;
-        default:
-            tc_phase_kernel<PH_FINAL><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, status);
-            break;
+        case PH_GRAM: e = launch_phase<PH_GRAM>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, st, sms); break;
+        case PH_POLY: e = launch_phase<PH_POLY>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, st, sms); break;
+        case PH_APPLY: e = launch_phase<PH_APPLY>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, st, sms); break;
+        default: e = launch_phase<PH_FINAL>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, st, sms); break;
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
