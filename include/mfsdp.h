@@ -167,8 +167,8 @@ int mfsdp_muon_workspace_size(const mfsdp_matrix* mats, int32_t n, const mfsdp_m
  * Alignment: param/grad aligned to their element size, momentum and
  * update_out to 4 bytes (16-byte alignment enables vector access).  Matrices
  * must not alias one another.  Launches: one momentum kernel, one norm kernel,
- * three GEMM-phase kernels per Newton-Schulz iteration (the last also writes W),
- * or one write kernel when ns_steps = 0.
+ * three GEMM-phase kernels per Newton-Schulz iteration, one parameter-write
+ * kernel.
  * Errors: MFSDP_ERR_INVALID_ARG, MFSDP_ERR_UNSUPPORTED_DTYPE, MFSDP_ERR_MISALIGNED,
  * MFSDP_ERR_WORKSPACE_TOO_SMALL, MFSDP_ERR_UNSUPPORTED_DEVICE, MFSDP_ERR_CUDA.
  */
@@ -236,9 +236,10 @@ int mfsdp_adamw_tail(float* p, const float* g, float* m, float* v, int64_t n,
 #define MFSDP_KCLASS_NORM      1   /* Frobenius norm finalisation */
 #define MFSDP_KCLASS_GRAM      2   /* A = X X^T */
 #define MFSDP_KCLASS_POLY      3   /* B = b A + c A A */
-#define MFSDP_KCLASS_APPLY     4   /* X <- a X + B X (and the final write) */
-#define MFSDP_KCLASS_WRITE0    5   /* parameter write when ns_steps = 0 */
+#define MFSDP_KCLASS_APPLY     4   /* X <- a X + B X */
+#define MFSDP_KCLASS_WRITE     5   /* parameter write: W <- W (1 - lr wd) - lr O */
 #define MFSDP_KCLASS_ADAMW     6   /* AdamW tail */
+#define MFSDP_KCLASS_FINAL     7   /* last iteration's X <- a X + B X (fp32 master only) */
 #define MFSDP_KCLASS_COUNT     8
 
 typedef struct {

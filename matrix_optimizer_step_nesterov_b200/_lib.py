@@ -40,7 +40,7 @@ EXPORTED = (
     "mfsdp_profile_begin", "mfsdp_profile_end", "mfsdp_muon_step_noalloc",
 )
 
-KCLASS_NAMES = ("momentum", "norm", "gram", "poly", "apply", "write0", "adamw", "unused")
+KCLASS_NAMES = ("momentum", "norm", "gram", "poly", "apply", "write", "adamw", "final")
 
 
 class MfsdpError(RuntimeError):

@@ -261,7 +261,7 @@ extern "C" int mfsdp_muon_step_launches(const mfsdp_matrix* mats, int32_t n, con
     if (st) return st;
     int32_t live = 0;
     for (int32_t i = 0; i < n; ++i) live += (mats[i].rows > 0 && mats[i].cols > 0);
-    *launches = live == 0 ? 0 : 2 + (hp->ns_steps == 0 ? 1 : 3 * hp->ns_steps);
+    *launches = live == 0 ? 0 : 3 + 3 * hp->ns_steps;
     return MFSDP_OK;
 }
 
@@ -340,12 +340,6 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     e = launch_norm(d_mats, nm, d_partials, d_s, hp->eps, s);
     prof_after(slot, s);
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
-    if (hp->ns_steps == 0) {
-        slot = prof_before(MFSDP_KCLASS_WRITE0, s);
-        e = launch_write0(d_mats, nm, L.mom_tiles, sc, d_s, s);
-        prof_after(slot, s);
-        return e == cudaSuccess ? MFSDP_OK : MFSDP_ERR_CUDA;
-    }
     const int32_t nsym = static_cast<int32_t>(L.sym_tiles.size());
     const int32_t ngen = static_cast<int32_t>(L.gen_tiles.size());
     auto gemm = [&](Phase ph, const TileDev* tiles, int32_t ntiles, int32_t it, int cls) {
@@ -357,12 +351,19 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
         return r;
     };
     for (int32_t it = 0; it < hp->ns_steps; ++it) {
-        const Phase last = (it == hp->ns_steps - 1) ? PH_FINAL : PH_APPLY;
+        const bool last = it == hp->ns_steps - 1;
         e = gemm(PH_GRAM, d_sym, nsym, it, MFSDP_KCLASS_GRAM);
         if (e == cudaSuccess) e = gemm(PH_POLY, d_poly, nsym, it, MFSDP_KCLASS_POLY);
-        if (e == cudaSuccess) e = gemm(last, d_gen, ngen, it, MFSDP_KCLASS_APPLY);
+        if (e == cudaSuccess)
+            e = gemm(last ? PH_FINAL : PH_APPLY, d_gen, ngen, it, last ? MFSDP_KCLASS_FINAL : MFSDP_KCLASS_APPLY);
         if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     }
+    // the parameter write reads X from the fp32 master the last iteration wrote
+    const int32_t xsel = (hp->mode == MFSDP_MODE_BF16) ? 0 : (hp->ns_steps & 1);
+    slot = prof_before(MFSDP_KCLASS_WRITE, s);
+    e = launch_param_write(d_mats, nm, L.mom_tiles, sc, d_s, xsel, hp->ns_steps == 0 ? 1 : 0, s);
+    prof_after(slot, s);
+    if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     return MFSDP_OK;
 }
 

@@ -98,23 +98,32 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     float sumsq = 0.f;
 
     if (full && md.mom_vec) {
+        // all eight 16-byte loads of this thread are issued before any store
+        float4 b[4], g[4];
+        int64_t idx[4];
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            idx[e] = (i0 + (v >> 4)) * cols + j0 + (v & 15) * 4;
+            b[e] = __ldcs(reinterpret_cast<const float4*>(md.buf + idx[e]));
+            g[e] = load4(md.grad, idx[e], gbf);
+        }
         #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int v = e * 256 + threadIdx.x;
             const int row = v >> 4, col = (v & 15) * 4;
-            const int64_t idx = (i0 + row) * cols + j0 + col;
-            float4 b = *reinterpret_cast<const float4*>(md.buf + idx);
-            const float4 g = load4(md.grad, idx, gbf);
+            float4 bb = b[e];
+            const float4 gg = g[e];
             float4 m;
-            b.x = beta * b.x + omb * g.x;  b.y = beta * b.y + omb * g.y;
-            b.z = beta * b.z + omb * g.z;  b.w = beta * b.w + omb * g.w;
+            bb.x = beta * bb.x + omb * gg.x;  bb.y = beta * bb.y + omb * gg.y;
+            bb.z = beta * bb.z + omb * gg.z;  bb.w = beta * bb.w + omb * gg.w;
             if (sc.nesterov) {
-                m.x = omb * g.x + beta * b.x;  m.y = omb * g.y + beta * b.y;
-                m.z = omb * g.z + beta * b.z;  m.w = omb * g.w + beta * b.w;
+                m.x = omb * gg.x + beta * bb.x;  m.y = omb * gg.y + beta * bb.y;
+                m.z = omb * gg.z + beta * bb.z;  m.w = omb * gg.w + beta * bb.w;
             } else {
-                m = b;
+                m = bb;
             }
-            *reinterpret_cast<float4*>(md.buf + idx) = b;
+            __stcs(reinterpret_cast<float4*>(md.buf + idx[e]), bb);
             sumsq += m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
             if (!tr) {
                 const int64_t xi = (i0 + row) * ldx + j0 + col;
@@ -148,15 +157,28 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     }
     if (tr) {
         __syncthreads();
-        // X = M^T: X[j][i] = M[i][j]; consecutive threads write consecutive i.
-        for (int e = 0; e < 16; ++e) {
-            const int v = e * 256 + threadIdx.x;
-            const int orow = v >> 6, ocol = v & 63;   // X row = M col, X col = M row
-            const int64_t xr = j0 + orow, xc = i0 + ocol;
-            if (xr < cols && xc < rows) {
-                const float m = tileM[ocol][orow];
-                xf[xr * ldx + xc] = m;
-                if (bf16_mode) xb[xr * ldx + xc] = __float2bfloat16_rn(m);
+        // X = M^T: X[j][i] = M[i][j]; a thread writes 4 consecutive i of one X row
+        if (full && md.mom_vec) {
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int v = e * 256 + threadIdx.x;
+                const int orow = v >> 4, oc = (v & 15) * 4;     // X row = M col, X cols oc..oc+3 = M rows
+                const float4 m = make_float4(tileM[oc][orow], tileM[oc + 1][orow], tileM[oc + 2][orow],
+                                             tileM[oc + 3][orow]);
+                const int64_t xi = (j0 + orow) * ldx + i0 + oc;
+                *reinterpret_cast<float4*>(xf + xi) = m;
+                if (bf16_mode) store4_bf16(xb, xi, m);
+            }
+        } else {
+            for (int e = 0; e < 16; ++e) {
+                const int v = e * 256 + threadIdx.x;
+                const int orow = v >> 6, ocol = v & 63;   // X row = M col, X col = M row
+                const int64_t xr = j0 + orow, xc = i0 + ocol;
+                if (xr < cols && xc < rows) {
+                    const float m = tileM[ocol][orow];
+                    xf[xr * ldx + xc] = m;
+                    if (bf16_mode) xb[xr * ldx + xc] = __float2bfloat16_rn(m);
+                }
             }
         }
     }
@@ -179,31 +201,77 @@ norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict_
     if (threadIdx.x == 0) s_out[mi] = (float)(1.0 / (sqrt(tot) + (double)eps));
 }
 
-// ns_steps = 0: O = scale * s * M, W <- W decay - lr O (same tiling as K1).
+// Parameter write, one 64 x 64 tile of W per block (the momentum tiling):
+//   O = f * X (transposed back when rows > cols),  W <- W (1 - lr wd) - lr O
+// with f = shape scale, times s when no Newton-Schulz iteration ran (X is then
+// the unnormalised M).  X comes from the fp32 master buffer `xsel`.  A
+// transposed X tile goes through shared memory so both X and W are read and
+// written along their rows; full tiles move 4 elements per access.
 __global__ void __launch_bounds__(256)
-write0_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, const float* __restrict__ s) {
+param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, const float* __restrict__ s,
+                   int xsel, int use_s, int32_t* status) {
+    __shared__ float tileX[kMomTile][kMomTile + 1];
     const int tile = blockIdx.x;
     const int mi = find_matrix(mats, nmats, tile);
     const MatDev& md = mats[mi];
     const int local = tile - md.mom_tile0;
+    const int64_t rows = md.rows, cols = md.cols;
     const int ti = local / md.mom_tiles_n, tj = local % md.mom_tiles_n;
-    const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;
-    const float f = md.shape_scale * s[mi];
+    if (local < 0 || ti >= (rows + kMomTile - 1) / kMomTile) {
+        record_status(status, -7);
+        return;
+    }
+    const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;   // W tile origin
+    const float f = md.shape_scale * (use_s ? s[mi] : 1.0f);
+    const float lr = sc.lr, decay = sc.decay;
+    const float* __restrict__ xf = md.xf[xsel];
+    const int64_t ldx = md.ldx;
+    const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
+    const bool wbf = md.param_bf16 != 0;
+    float* wf = static_cast<float*>(md.param);
+    __nv_bfloat16* wb = static_cast<__nv_bfloat16*>(md.param);
+    float* uo = md.update_out;
+    if (md.tr) {
+        // X tile rows = W columns j0.., X tile columns = W rows i0..
+        for (int e = 0; e < 16; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            const int xr = v >> 6, xc = v & 63;
+            if (j0 + xr < cols && i0 + xc < rows) tileX[xr][xc] = xf[(j0 + xr) * ldx + i0 + xc];
+        }
+        __syncthreads();
+    }
+    const bool vec = full && (cols % 4 == 0) && (reinterpret_cast<uintptr_t>(md.param) % (wbf ? 8 : 16) == 0) &&
+                     (uo == nullptr || reinterpret_cast<uintptr_t>(uo) % 16 == 0);
+    if (vec) {
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            const int row = v >> 4, col = (v & 15) * 4;
+            const int64_t widx = (i0 + row) * cols + j0 + col;
+            float4 x;
+            if (md.tr) x = make_float4(tileX[col][row], tileX[col + 1][row], tileX[col + 2][row], tileX[col + 3][row]);
+            else x = *reinterpret_cast<const float4*>(xf + (i0 + row) * ldx + j0 + col);
+            float4 w = load4(md.param, widx, wbf);
+            const float4 o = make_float4(f * x.x, f * x.y, f * x.z, f * x.w);
+            w.x = fmaf(-lr, o.x, w.x * decay); w.y = fmaf(-lr, o.y, w.y * decay);
+            w.z = fmaf(-lr, o.z, w.z * decay); w.w = fmaf(-lr, o.w, w.w * decay);
+            if (wbf) store4_bf16(wb, widx, w);
+            else *reinterpret_cast<float4*>(wf + widx) = w;
+            if (uo) *reinterpret_cast<float4*>(uo + widx) = o;
+        }
+        return;
+    }
     for (int e = 0; e < 16; ++e) {
         const int v = e * 256 + threadIdx.x;
-        const int64_t i = i0 + (v >> 6), j = j0 + (v & 63);
-        if (i >= md.rows || j >= md.cols) continue;
-        const float x = md.tr ? md.xf[0][j * md.ldx + i] : md.xf[0][i * md.ldx + j];
+        const int row = v >> 6, col = v & 63;
+        const int64_t i = i0 + row, j = j0 + col;
+        if (i >= rows || j >= cols) continue;
+        const float x = md.tr ? tileX[col][row] : xf[i * ldx + j];
         const float o = f * x;
-        const int64_t idx = i * md.cols + j;
-        if (md.update_out) md.update_out[idx] = o;
-        if (md.param_bf16) {
-            __nv_bfloat16* w = static_cast<__nv_bfloat16*>(md.param);
-            w[idx] = __float2bfloat16_rn(fmaf(-sc.lr, o, __bfloat162float(w[idx]) * sc.decay));
-        } else {
-            float* w = static_cast<float*>(md.param);
-            w[idx] = fmaf(-sc.lr, o, w[idx] * sc.decay);
-        }
+        const int64_t idx = i * cols + j;
+        if (uo) uo[idx] = o;
+        if (wbf) wb[idx] = __float2bfloat16_rn(fmaf(-lr, o, __bfloat162float(wb[idx]) * decay));
+        else wf[idx] = fmaf(-lr, o, wf[idx] * decay);
     }
 }
 
@@ -281,10 +349,10 @@ cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partia
     return cudaGetLastError();
 }
 
-cudaError_t launch_write0(const MatDev* d_mats, int32_t nmats, int32_t total_tiles,
-                          const StepScalars& sc, const float* s, cudaStream_t st) {
+cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_tiles, const StepScalars& sc,
+                               const float* s, int32_t xsel, int32_t use_s, cudaStream_t st) {
     if (total_tiles <= 0) return cudaSuccess;
-    write0_kernel<<<total_tiles, 256, 0, st>>>(d_mats, nmats, sc, s);
+    param_write_kernel<<<total_tiles, 256, 0, st>>>(d_mats, nmats, sc, s, xsel, use_s, device_status_ptr());
     return cudaGetLastError();
 }
 

@@ -7,7 +7,7 @@
 //   PH_GRAM   A = s^2 X X^T       upper-triangle tiles, mirrored store
 //   PH_POLY   B = b A + c A A     upper-triangle tiles, mirrored store (A symmetric, so A A = A A^T)
 //   PH_APPLY  X <- s (a X + B X)
-//   PH_FINAL  O = scale s (a X + B X);  W <- W (1 - lr wd) - lr O
+//   PH_FINAL  the same X update into the fp32 master only (the parameter write follows)
 // in the diagonal-split form of internal.h: the GEMM operands are the
 // zero-diagonal parts E_A, E_B; the diagonals d_A, d_B enter in fp32 epilogues.
 // s is the Frobenius scale 1/(||M||+eps) on the first iteration and 1 after:
@@ -214,24 +214,11 @@ simt_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, int32_t nmats,
                 const int64_t xi = (int64_t)gi * md.ldx + gj;
                 const float xin = md.xf[BF16 ? 0 : cur][xi];
                 const float v = sg * fmaf(sc.a + md.db[gi], xin, a);
-                if (ph == PH_APPLY) {
-                    if (BF16) {
-                        md.xf[0][xi] = v;
-                        md.xb[nxt][xi] = __float2bfloat16_rn(v);
-                    } else {
-                        md.xf[nxt][xi] = v;
-                    }
+                if (BF16) {
+                    md.xf[0][xi] = v;
+                    if (ph == PH_APPLY) md.xb[nxt][xi] = __float2bfloat16_rn(v);
                 } else {
-                    const float o = md.shape_scale * v;
-                    const int64_t widx = md.tr ? (int64_t)gj * md.cols + gi : (int64_t)gi * md.cols + gj;
-                    if (md.update_out) md.update_out[widx] = o;
-                    if (md.param_bf16) {
-                        __nv_bfloat16* w = static_cast<__nv_bfloat16*>(md.param);
-                        w[widx] = __float2bfloat16_rn(fmaf(-sc.lr, o, __bfloat162float(w[widx]) * sc.decay));
-                    } else {
-                        float* w = static_cast<float*>(md.param);
-                        w[widx] = fmaf(-sc.lr, o, w[widx] * sc.decay);
-                    }
+                    md.xf[nxt][xi] = v;
                 }
             }
         }

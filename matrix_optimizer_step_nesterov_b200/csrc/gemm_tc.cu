@@ -238,7 +238,7 @@ __host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major, int m) {
 }
 
 // ---------------------------------------------------------------------------
-// Warp-cooperative epilogue of one 32 x 32 chunk of the accumulator.
+// Warp-cooperative GRAM / POLY epilogue of one 32 x 32 chunk of the accumulator.
 // TMEM delivers it in the row domain: lane l holds row gi0 + l, columns
 // gj0 .. gj0 + 31.  Accesses that run along a column (the mirrored triangle
 // of a symmetric result, the transposed parameter write) are issued straight
@@ -319,120 +319,54 @@ __device__ __forceinline__ void epilogue_chunk_warp(const MatDev& md, int iter, 
         __syncwarp();
         return;
     }
-    // APPLY / FINAL: X_new = s ((a + d_B,i) X + E_B X), computed in the column domain
-    float* xf = md.xf[0];
-    const int64_t ldx = md.ldx;
-    #pragma unroll
-    for (int t = 0; t < 32; ++t) stg[lane][t] = __uint_as_float(r[t]);
-    const float fa = row_ok ? (sc.a + md.db[gi]) : 0.f;
-    __syncwarp();
-    if (ph == PH_APPLY) {
-        __nv_bfloat16* xbn = md.xb[nxt];
-        const float* xcol = xf + (int64_t)gi0 * ldx + gjc;
-        #pragma unroll 1
-        for (int h = 0; h < 32; h += 16) {          // 16 loads in flight per lane
-            float xv[16];
-            #pragma unroll
-            for (int k = 0; k < 16; ++k)
-                xv[k] = (gi0 + h + k < Mrows && col_ok) ? xcol[(int64_t)(h + k) * ldx] : 0.f;
-            #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int rr = h + k;
-                const float f = __shfl_sync(0xffffffffu, fa, rr);
-                if (gi0 + rr < Mrows && col_ok) {
-                    const int64_t idx = (int64_t)(gi0 + rr) * ldx + gjc;
-                    const float v = sg * fmaf(f, xv[k], stg[rr][lane]);
-                    xf[idx] = v;
-                    xbn[idx] = __float2bfloat16_rn(v);
-                }
-            }
-        }
-        __syncwarp();
-        return;
-    }
-    float xv[32];
-    #pragma unroll
-    for (int rr = 0; rr < 32; ++rr) {
-        const int gi2 = gi0 + rr;
-        xv[rr] = (gi2 < Mrows && col_ok) ? xf[(int64_t)gi2 * ldx + gjc] : 0.f;
-    }
-    // FINAL: O = scale * X_new, W <- W (1 - lr wd) - lr O, at W[i][j] or, transposed, W[j][i]
-    const int64_t cols = md.cols;
-    #pragma unroll
-    for (int rr = 0; rr < 32; ++rr) {
-        const float f = __shfl_sync(0xffffffffu, fa, rr);
-        xv[rr] = md.shape_scale * (sg * fmaf(f, xv[rr], stg[rr][lane]));   // O, column domain
-    }
-    if (!md.tr) {
-        float wv[32];
-        #pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-            const int gi2 = gi0 + rr;
-            const int64_t widx = (int64_t)gi2 * cols + gjc;
-            wv[rr] = 0.f;
-            if (gi2 < Mrows && col_ok)
-                wv[rr] = md.param_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(md.param)[widx])
-                                       : static_cast<const float*>(md.param)[widx];
-        }
-        #pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-            const int gi2 = gi0 + rr;
-            if (gi2 < Mrows && col_ok) {
-                const int64_t widx = (int64_t)gi2 * cols + gjc;
-                const float o = xv[rr];
-                if (md.update_out) md.update_out[widx] = o;
-                const float w = fmaf(-sc.lr, o, wv[rr] * sc.decay);
-                if (md.param_bf16) static_cast<__nv_bfloat16*>(md.param)[widx] = __float2bfloat16_rn(w);
-                else static_cast<float*>(md.param)[widx] = w;
-            }
-        }
-        __syncwarp();
-        return;
-    }
-    // transposed parameter: back to the row domain, W[j][i] consecutive across lanes
-    #pragma unroll
-    for (int rr = 0; rr < 32; ++rr) stg[rr][lane] = xv[rr];
-    __syncwarp();
-    float wv[32];
-    #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-        const int gj = gj0 + t;
-        const int64_t widx = (int64_t)gj * cols + gi;
-        wv[t] = 0.f;
-        if (row_ok && gj < Ncols)
-            wv[t] = md.param_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(md.param)[widx])
-                                  : static_cast<const float*>(md.param)[widx];
-    }
-    #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-        const int gj = gj0 + t;
-        if (row_ok && gj < Ncols) {
-            const int64_t widx = (int64_t)gj * cols + gi;
-            const float o = stg[lane][t];
-            if (md.update_out) md.update_out[widx] = o;
-            const float w = fmaf(-sc.lr, o, wv[t] * sc.decay);
-            if (md.param_bf16) static_cast<__nv_bfloat16*>(md.param)[widx] = __float2bfloat16_rn(w);
-            else static_cast<float*>(md.param)[widx] = w;
-        }
-    }
-    __syncwarp();
 }
 
-// APPLY epilogue of one warp over its chunks [qa, qb) of a tile, software
-// pipelined: the 16 master-X loads of the next half-chunk are issued before
-// the current half-chunk is computed and stored, so global latency overlaps
-// the stores and the TMEM reads.
-__device__ __forceinline__ void epilogue_apply_warp(const MatDev& md, int iter, const StepScalars& sc, float sg,
-                                                    int gi0, int gj_tile, int qa, int qb, int Mrows, int Ncols,
-                                                    uint32_t trow, float (*stg)[33], int lane) {
-    const int nxt = (iter & 1) ^ 1;
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+}
+
+// L2 prefetch of a warp's block of a row-major matrix: rows [r0, r0 + nr) of
+// width `row_bytes` starting `col_byte0` bytes into each row, one 128-byte
+// line per lane per round.  Addresses stay inside the named rows.
+__device__ __forceinline__ void prefetch_block(const void* base, int64_t ld_bytes, int r0, int nr, int64_t col_byte0,
+                                               int64_t row_bytes, int lane) {
+    if (nr <= 0 || row_bytes <= 0) return;
+    const int lines = (int)((row_bytes + 127) / 128);
+    const char* b = static_cast<const char*>(base);
+    for (int i = lane; i < nr * lines; i += 32) {
+        const int rr = i / lines, ln = i - rr * lines;
+        prefetch_l2(b + (int64_t)(r0 + rr) * ld_bytes + col_byte0 + (int64_t)ln * 128);
+    }
+}
+
+// The fp32 master-X block the APPLY / FINAL epilogue of a tile reads, fetched
+// into L2 while the warp still waits for the accumulator.
+template <int ph>
+__device__ __forceinline__ void prefetch_tile_operands(const MatDev& md, int gi0, int gjb, int Mrows, int Ncols,
+                                                       int lane) {
+    if (ph != PH_APPLY && ph != PH_FINAL) return;
+    const int nr = min(32, Mrows - gi0);
+    const int nc = min(BN / 2, Ncols - gjb);
+    if (nr <= 0 || nc <= 0) return;
+    prefetch_block(md.xf[0], md.ldx * 4, gi0, nr, (int64_t)gjb * 4, (int64_t)nc * 4, lane);
+}
+
+// APPLY / FINAL epilogue of one warp over its chunks [qa, qb) of a tile:
+//   X <- s ((a + d_B,i) X + E_B X) into the fp32 master, plus (APPLY) the bf16
+//   operand copy the next iteration's GEMMs read.
+// X is read in the column domain (coalesced along its rows), 16 rows at a
+// time, and the loads of the next 16 rows are issued before the current ones
+// are computed and stored.
+template <int ph>
+__device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, const StepScalars& sc, float sg,
+                                                int gi0, int gj_tile, int qa, int qb, int Mrows, int Ncols,
+                                                uint32_t trow, float (*stg)[33], int lane) {
     float* xf = md.xf[0];
-    __nv_bfloat16* xbn = md.xb[nxt];
+    __nv_bfloat16* xbn = md.xb[(iter & 1) ^ 1];
     const int64_t ldx = md.ldx;
     const int gi = gi0 + lane;
     const float fa = gi < Mrows ? (sc.a + md.db[gi]) : 0.f;
-    // chunks [qa, qe) hold at least one column in range (rows checked by the caller)
-    int qe = qa;
+    int qe = qa;                                  // chunks [qa, qe) hold a column in range
     while (qe < qb && gj_tile + qe * 32 < Ncols) ++qe;
     const int nb = 2 * (qe - qa);                 // half-chunks of 16 rows
     if (nb == 0) return;
@@ -471,7 +405,7 @@ __device__ __forceinline__ void epilogue_apply_warp(const MatDev& md, int iter, 
                     const int64_t idx = (int64_t)(gi0 + rr) * ldx + gjc;
                     const float v = sg * fmaf(fk[k], cur[k], stg[rr][lane]);
                     xf[idx] = v;
-                    xbn[idx] = __float2bfloat16_rn(v);
+                    if (ph == PH_APPLY) xbn[idx] = __float2bfloat16_rn(v);
                 }
             }
         }
@@ -664,21 +598,30 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
         uint32_t acc_phase = 0;
         for (int t = cluster_id; t < ntiles; t += nclusters) {
             const TileDev td = tiles[t];
-            const MatDev& md = mats[td.mat];
+            const MatDev md = mats[td.mat];   // a register copy: global stores below cannot alias it
             const int Mrows = md.r;
             const int Ncols = gemm ? md.c : md.r;
+            const int gi0 = td.tm * C::TILE_M + (int)rank * BM + quad * 32;
+            // fetch the operands of this tile (first one only) and of the next into L2
+            // while the accumulator is still being computed
+            if (t == cluster_id) prefetch_tile_operands<ph>(md, gi0, td.tn * BN + half * (BN / 2), Mrows, Ncols, lane);
+            if (t + nclusters < ntiles) {
+                const TileDev tn2 = tiles[t + nclusters];
+                const MatDev& m2 = mats[tn2.mat];
+                prefetch_tile_operands<ph>(m2, tn2.tm * C::TILE_M + (int)rank * BM + quad * 32,
+                                           tn2.tn * BN + half * (BN / 2), m2.r, gemm ? m2.c : m2.r, lane);
+            }
             bool ok = true;
             if (lane == 0) ok = wait_bounded(tfull0 + 8 * acc, acc_phase, abort_flag, status);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
             tc_fence_after();
             const float sg = (iter == 0) ? s[td.mat] : 1.0f;
-            const int gi0 = td.tm * C::TILE_M + (int)rank * BM + quad * 32;
             const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
             float (*stg)[33] = reinterpret_cast<float (*)[33]>(stg_all + (warp - 2) * 32 * 33);
-            if constexpr (ph == PH_APPLY) {
+            if constexpr (ph == PH_APPLY || ph == PH_FINAL) {
                 if (gi0 < Mrows)
-                    epilogue_apply_warp(md, iter, sc, sg, gi0, td.tn * BN, half * (BN / 64), (half + 1) * (BN / 64),
+                    epilogue_x_warp<ph>(md, iter, sc, sg, gi0, td.tn * BN, half * (BN / 64), (half + 1) * (BN / 64),
                                         Mrows, Ncols, trow, stg, lane);
             } else {
                 #pragma unroll 1

@@ -55,8 +55,9 @@ struct TileDev {
 enum Phase : int32_t {
     PH_GRAM = 0,   // A = s^2 X X^T -> E_A (fp32 + operand copy), d_A   (upper tiles, mirrored)
     PH_POLY = 1,   // B = b A + c A A -> E_B operand, d_B                (upper tiles, mirrored)
-    PH_APPLY = 2,  // X <- s ((a + d_B,i) X + E_B X)
-    PH_FINAL = 3,  // last iteration: O = scale * X_new; W <- W (1 - lr wd) - lr O
+    PH_APPLY = 2,  // X <- s ((a + d_B,i) X + E_B X)   (fp32 master + bf16 operand copy)
+    PH_FINAL = 3,  // last iteration: the same X update into the fp32 master only; the
+                   // parameter write then runs as its own HBM-bound kernel
 };
 
 struct StepScalars {
@@ -83,8 +84,9 @@ cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_t
                             const StepScalars& sc, float* partials, cudaStream_t st);
 cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partials,
                         float* s_out, float eps, cudaStream_t st);
-cudaError_t launch_write0(const MatDev* d_mats, int32_t nmats, int32_t total_tiles,
-                          const StepScalars& sc, const float* s, cudaStream_t st);
+// W <- W (1 - lr wd) - lr * scale * (use_s ? s : 1) * X, X from the fp32 master xf[xsel]
+cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_tiles, const StepScalars& sc,
+                               const float* s, int32_t xsel, int32_t use_s, cudaStream_t st);
 cudaError_t launch_gemm_simt(Phase ph, const MatDev* d_mats, int32_t nmats, const TileDev* d_tiles, int32_t ntiles,
                              int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st);
 cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, int64_t n,

@@ -159,7 +159,7 @@ def test_empty_step_is_a_noop_without_a_device(lib):
 
 def test_launch_count(lib):
     hp = lib.muon_hparams()
-    assert lib.mfsdp_muon_step_launches([_mat(lib, 64, 64)], hp) == 2 + 3 * 5
+    assert lib.mfsdp_muon_step_launches([_mat(lib, 64, 64)], hp) == 3 + 3 * 5
     assert lib.mfsdp_muon_step_launches([_mat(lib, 64, 64)], lib.muon_hparams(ns_steps=0)) == 3
     assert lib.mfsdp_muon_step_launches([], hp) == 0
 
