@@ -76,16 +76,30 @@ def ns_flops_dense(specs, steps: int = 5) -> float:
 
 
 def split_groups(specs, n_groups: int) -> List[List[int]]:
-    """Contiguous groups of matrix indices with about equal dense NS FLOPs."""
+    """Matrix-index groups for the pipelined e2e measurement.  With three or
+    more groups the first and the last hold a single small matrix, so that the
+    copies nothing overlaps (the first group's upload, the last group's
+    download) stay short; the matrices between are split into groups of about
+    equal dense NS FLOPs."""
     costs = [ns_flops_dense([s]) for s in specs]
-    total = sum(costs)
-    groups: List[List[int]] = [[] for _ in range(n_groups)]
+    order = list(range(len(specs)))
+    if n_groups >= 3 and len(specs) >= n_groups:
+        by_size = sorted(order, key=lambda i: (costs[i], i))
+        first, last = by_size[0], by_size[1]
+        middle = [i for i in order if i not in (first, last)]
+        return [[first]] + _balanced(middle, costs, n_groups - 2) + [[last]]
+    return _balanced(order, costs, n_groups)
+
+
+def _balanced(idx: List[int], costs: List[float], n_groups: int) -> List[List[int]]:
+    total = sum(costs[i] for i in idx)
+    groups: List[List[int]] = [[] for _ in range(max(1, n_groups))]
     acc, g = 0.0, 0
-    for i, c in enumerate(costs):
-        if g < n_groups - 1 and groups[g] and acc + c / 2 > total * (g + 1) / n_groups:
+    for i in idx:
+        if g < len(groups) - 1 and groups[g] and acc + costs[i] / 2 > total * (g + 1) / len(groups):
             g += 1
         groups[g].append(i)
-        acc += c
+        acc += costs[i]
     return [grp for grp in groups if grp]
 
 
@@ -558,7 +572,7 @@ def main(argv=None) -> int:
     ap.add_argument("--tail", type=int, default=0, help="tail length with --shapes")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-groups", type=int, default=4, help="matrix groups pipelined in the e2e measurement")
+    ap.add_argument("--e2e-groups", type=int, default=6, help="matrix groups pipelined in the e2e measurement")
     ap.add_argument("--no-tail-bench", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")

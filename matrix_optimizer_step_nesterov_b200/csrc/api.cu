@@ -116,6 +116,7 @@ struct Layout {
     std::vector<TileDev> poly_tiles;   // PH_POLY
     std::vector<TileDev> gen_tiles;    // PH_APPLY / PH_FINAL
     int32_t mom_tiles = 0;
+    int32_t mom_groups = 0;
     size_t off_mats = 0, off_maps = 0, off_sym = 0, off_poly = 0, off_gen = 0, off_partials = 0, off_s = 0;
     size_t head_end = 0, maps_bytes = 0;
     size_t total = 0;
@@ -146,7 +147,7 @@ int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp
     const bool bf16 = hp->mode == MFSDP_MODE_BF16;
     L.engine = pick_engine(hp);
     L.mats.clear();
-    int32_t tile0 = 0;
+    int32_t tile0 = 0, grp0 = 0;
     for (int32_t i = 0; i < n; ++i) {
         const mfsdp_matrix& u = in[i];
         if (u.rows == 0 || u.cols == 0) continue;
@@ -169,12 +170,15 @@ int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp
         const int64_t tiles = ((u.rows + kMomTile - 1) / kMomTile) * m.mom_tiles_n;
         if (tile0 + tiles > (1LL << 31) - 1) return MFSDP_ERR_INVALID_ARG;
         tile0 += static_cast<int32_t>(tiles);
+        m.mom_grp0 = grp0;
+        grp0 += static_cast<int32_t>((tiles + kMomGroup - 1) / kMomGroup);
         m.mom_vec = (u.cols % 4 == 0) && aligned(u.momentum, 16) &&
                     aligned(u.grad, u.grad_dtype == MFSDP_DTYPE_BF16 ? 8 : 16);
         m.shape_scale = static_cast<float>(std::sqrt(std::max(1.0, static_cast<double>(u.rows) / u.cols)));
         L.mats.push_back(m);
     }
     L.mom_tiles = tile0;
+    L.mom_groups = grp0;
     build_tiles(L, L.engine);
     const size_t nm = L.mats.size();
     size_t off = 0;
@@ -333,7 +337,7 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     sc.bf16_mode = hp->mode == MFSDP_MODE_BF16;
 
     int slot = prof_before(MFSDP_KCLASS_MOMENTUM, s);
-    cudaError_t e = launch_momentum(d_mats, nm, L.mom_tiles, sc, d_partials, s);
+    cudaError_t e = launch_momentum(d_mats, nm, L.mom_groups, sc, d_partials, s);
     prof_after(slot, s);
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     slot = prof_before(MFSDP_KCLASS_NORM, s);
@@ -361,7 +365,7 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     // the parameter write reads X from the fp32 master the last iteration wrote
     const int32_t xsel = (hp->mode == MFSDP_MODE_BF16) ? 0 : (hp->ns_steps & 1);
     slot = prof_before(MFSDP_KCLASS_WRITE, s);
-    e = launch_param_write(d_mats, nm, L.mom_tiles, sc, d_s, xsel, hp->ns_steps == 0 ? 1 : 0, s);
+    e = launch_param_write(d_mats, nm, L.mom_groups, sc, d_s, xsel, hp->ns_steps == 0 ? 1 : 0, s);
     prof_after(slot, s);
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     return MFSDP_OK;

@@ -41,12 +41,12 @@ __device__ __forceinline__ void store4_bf16(__nv_bfloat16* p, int64_t i, float4 
     *reinterpret_cast<uint2*>(p + i) = raw;
 }
 
-// index of the matrix owning momentum tile `tile` (largest i with mom_tile0 <= tile)
-__device__ __forceinline__ int find_matrix(const MatDev* mats, int nmats, int tile) {
+// index of the matrix owning tile group `grp` (largest i with mom_grp0 <= grp)
+__device__ __forceinline__ int find_matrix(const MatDev* mats, int nmats, int grp) {
     int lo = 0, hi = nmats - 1;
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
-        if (mats[mid].mom_tile0 <= tile) lo = mid; else hi = mid - 1;
+        if (mats[mid].mom_grp0 <= grp) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
@@ -72,22 +72,29 @@ __device__ __forceinline__ T block_sum(T v, T* smem) {
 // writes buf, the fp32 master X (M, or M^T when rows > cols) and, in bf16
 // mode, its bf16 operand copy; each tile's sum of M^2 goes to partials[tile].
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
                 float* __restrict__ partials, int32_t* status) {
     __shared__ float tileM[kMomTile][kMomTile + 1];
     __shared__ float red[8];
-    const int tile = blockIdx.x;
-    const int mi = find_matrix(mats, nmats, tile);
+    const int grp = blockIdx.x;
+    const int mi = find_matrix(mats, nmats, grp);
     const MatDev& md = mats[mi];
-    const int local = tile - md.mom_tile0;
     const int64_t rows = md.rows, cols = md.cols;
     const int64_t tiles_m = (rows + kMomTile - 1) / kMomTile;
-    const int ti = local / md.mom_tiles_n, tj = local % md.mom_tiles_n;
-    if (local < 0 || ti >= tiles_m) {  // cannot happen with a host-built table
+    // fields used inside the tile loop, read once (the loop's stores could otherwise force reloads)
+    float* __restrict__ bufp = md.buf;
+    const void* gradp = md.grad;
+    const int mom_vec = md.mom_vec, tiles_n = md.mom_tiles_n, tile0 = md.mom_tile0, grp0 = md.mom_grp0;
+    const int64_t ntiles = tiles_m * md.mom_tiles_n;
+    if (grp < grp0) {  // cannot happen with a host-built table
         record_status(status, -7);
         return;
     }
+    for (int k = 0; k < kMomGroup; ++k) {
+    const int local = (grp - grp0) * kMomGroup + k;
+    if (local >= ntiles) break;      // block-uniform
+    const int ti = local / tiles_n, tj = local % tiles_n;
     const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;
     const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
     const float beta = sc.beta, omb = 1.0f - sc.beta;
@@ -97,7 +104,7 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     const int64_t ldx = md.ldx;
     float sumsq = 0.f;
 
-    if (full && md.mom_vec) {
+    if (full && mom_vec) {
         // all eight 16-byte loads of this thread are issued before any store
         float4 b[4], g[4];
         int64_t idx[4];
@@ -105,8 +112,8 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
         for (int e = 0; e < 4; ++e) {
             const int v = e * 256 + threadIdx.x;
             idx[e] = (i0 + (v >> 4)) * cols + j0 + (v & 15) * 4;
-            b[e] = __ldcs(reinterpret_cast<const float4*>(md.buf + idx[e]));
-            g[e] = load4(md.grad, idx[e], gbf);
+            b[e] = __ldcs(reinterpret_cast<const float4*>(bufp + idx[e]));
+            g[e] = load4(gradp, idx[e], gbf);
         }
         #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -123,7 +130,7 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
             } else {
                 m = bb;
             }
-            __stcs(reinterpret_cast<float4*>(md.buf + idx[e]), bb);
+            __stcs(reinterpret_cast<float4*>(bufp + idx[e]), bb);
             sumsq += m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
             if (!tr) {
                 const int64_t xi = (i0 + row) * ldx + j0 + col;
@@ -141,10 +148,10 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
             const int64_t i = i0 + row, j = j0 + col;
             if (i < rows && j < cols) {
                 const int64_t idx = i * cols + j;
-                const float g = load_elem(md.grad, idx, gbf);
-                const float b = beta * md.buf[idx] + omb * g;
+                const float g = load_elem(gradp, idx, gbf);
+                const float b = beta * bufp[idx] + omb * g;
                 const float m = sc.nesterov ? (omb * g + beta * b) : b;
-                md.buf[idx] = b;
+                bufp[idx] = b;
                 sumsq += m * m;
                 if (!tr) {
                     xf[i * ldx + j] = m;
@@ -158,7 +165,7 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     if (tr) {
         __syncthreads();
         // X = M^T: X[j][i] = M[i][j]; a thread writes 4 consecutive i of one X row
-        if (full && md.mom_vec) {
+        if (full && mom_vec) {
             #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int v = e * 256 + threadIdx.x;
@@ -183,7 +190,9 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
         }
     }
     const float tot = block_sum(sumsq, red);
-    if (threadIdx.x == 0) partials[tile] = tot;
+    if (threadIdx.x == 0) partials[tile0 + local] = tot;
+    __syncthreads();                 // red and tileM are reused by the next tile
+    }
 }
 
 // K2: s = 1 / (||M||_F + eps) per matrix; fixed-order fp64 sum of the tile partials.
@@ -207,71 +216,95 @@ norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict_
 // the unnormalised M).  X comes from the fp32 master buffer `xsel`.  A
 // transposed X tile goes through shared memory so both X and W are read and
 // written along their rows; full tiles move 4 elements per access.
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, const float* __restrict__ s,
                    int xsel, int use_s, int32_t* status) {
     __shared__ float tileX[kMomTile][kMomTile + 1];
-    const int tile = blockIdx.x;
-    const int mi = find_matrix(mats, nmats, tile);
+    const int grp = blockIdx.x;
+    const int mi = find_matrix(mats, nmats, grp);
     const MatDev& md = mats[mi];
-    const int local = tile - md.mom_tile0;
     const int64_t rows = md.rows, cols = md.cols;
-    const int ti = local / md.mom_tiles_n, tj = local % md.mom_tiles_n;
-    if (local < 0 || ti >= (rows + kMomTile - 1) / kMomTile) {
+    const int tiles_n = md.mom_tiles_n, grp0 = md.mom_grp0;
+    const int64_t ntiles = ((rows + kMomTile - 1) / kMomTile) * tiles_n;
+    if (grp < grp0) {
         record_status(status, -7);
         return;
     }
-    const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;   // W tile origin
+    const bool tr = md.tr != 0;
     const float f = md.shape_scale * (use_s ? s[mi] : 1.0f);
     const float lr = sc.lr, decay = sc.decay;
     const float* __restrict__ xf = md.xf[xsel];
     const int64_t ldx = md.ldx;
-    const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
     const bool wbf = md.param_bf16 != 0;
     float* wf = static_cast<float*>(md.param);
     __nv_bfloat16* wb = static_cast<__nv_bfloat16*>(md.param);
     float* uo = md.update_out;
-    if (md.tr) {
+    const bool aligned_w = (cols % 4 == 0) && (reinterpret_cast<uintptr_t>(md.param) % (wbf ? 8 : 16) == 0) &&
+                           (uo == nullptr || reinterpret_cast<uintptr_t>(uo) % 16 == 0);
+    for (int k = 0; k < kMomGroup; ++k) {
+    const int local = (grp - grp0) * kMomGroup + k;
+    if (local >= ntiles) break;      // block-uniform
+    const int ti = local / tiles_n, tj = local % tiles_n;
+    const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;   // W tile origin
+    const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
+    if (tr) {
         // X tile rows = W columns j0.., X tile columns = W rows i0..
-        for (int e = 0; e < 16; ++e) {
-            const int v = e * 256 + threadIdx.x;
-            const int xr = v >> 6, xc = v & 63;
-            if (j0 + xr < cols && i0 + xc < rows) tileX[xr][xc] = xf[(j0 + xr) * ldx + i0 + xc];
+        if (full && (ldx % 4 == 0)) {
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int v = e * 256 + threadIdx.x;
+                const int xr = v >> 4, xc = (v & 15) * 4;
+                const float4 x = *reinterpret_cast<const float4*>(xf + (j0 + xr) * ldx + i0 + xc);
+                tileX[xr][xc] = x.x; tileX[xr][xc + 1] = x.y; tileX[xr][xc + 2] = x.z; tileX[xr][xc + 3] = x.w;
+            }
+        } else {
+            for (int e = 0; e < 16; ++e) {
+                const int v = e * 256 + threadIdx.x;
+                const int xr = v >> 6, xc = v & 63;
+                if (j0 + xr < cols && i0 + xc < rows) tileX[xr][xc] = xf[(j0 + xr) * ldx + i0 + xc];
+            }
         }
         __syncthreads();
     }
-    const bool vec = full && (cols % 4 == 0) && (reinterpret_cast<uintptr_t>(md.param) % (wbf ? 8 : 16) == 0) &&
-                     (uo == nullptr || reinterpret_cast<uintptr_t>(uo) % 16 == 0);
-    if (vec) {
+    if (full && aligned_w) {
+        // every load of this thread is issued before any store
+        float4 xv[4], wv[4];
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            const int row = v >> 4, col = (v & 15) * 4;
+            if (tr) xv[e] = make_float4(tileX[col][row], tileX[col + 1][row], tileX[col + 2][row], tileX[col + 3][row]);
+            else xv[e] = *reinterpret_cast<const float4*>(xf + (i0 + row) * ldx + j0 + col);
+            wv[e] = load4(md.param, (i0 + row) * cols + j0 + col, wbf);
+        }
         #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int v = e * 256 + threadIdx.x;
             const int row = v >> 4, col = (v & 15) * 4;
             const int64_t widx = (i0 + row) * cols + j0 + col;
-            float4 x;
-            if (md.tr) x = make_float4(tileX[col][row], tileX[col + 1][row], tileX[col + 2][row], tileX[col + 3][row]);
-            else x = *reinterpret_cast<const float4*>(xf + (i0 + row) * ldx + j0 + col);
-            float4 w = load4(md.param, widx, wbf);
-            const float4 o = make_float4(f * x.x, f * x.y, f * x.z, f * x.w);
+            const float4 o = make_float4(f * xv[e].x, f * xv[e].y, f * xv[e].z, f * xv[e].w);
+            float4 w = wv[e];
             w.x = fmaf(-lr, o.x, w.x * decay); w.y = fmaf(-lr, o.y, w.y * decay);
             w.z = fmaf(-lr, o.z, w.z * decay); w.w = fmaf(-lr, o.w, w.w * decay);
             if (wbf) store4_bf16(wb, widx, w);
             else *reinterpret_cast<float4*>(wf + widx) = w;
             if (uo) *reinterpret_cast<float4*>(uo + widx) = o;
         }
-        return;
-    }
+    } else {
     for (int e = 0; e < 16; ++e) {
         const int v = e * 256 + threadIdx.x;
         const int row = v >> 6, col = v & 63;
         const int64_t i = i0 + row, j = j0 + col;
         if (i >= rows || j >= cols) continue;
-        const float x = md.tr ? tileX[col][row] : xf[i * ldx + j];
+        const float x = tr ? tileX[col][row] : xf[i * ldx + j];
         const float o = f * x;
         const int64_t idx = i * cols + j;
         if (uo) uo[idx] = o;
         if (wbf) wb[idx] = __float2bfloat16_rn(fmaf(-lr, o, __bfloat162float(wb[idx]) * decay));
         else wf[idx] = fmaf(-lr, o, wf[idx] * decay);
+    }
+    }
+    __syncthreads();                 // tileX is reused by the next tile
     }
 }
 
@@ -335,10 +368,10 @@ int sm_count() {
 
 }  // namespace
 
-cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_tiles,
+cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_groups,
                             const StepScalars& sc, float* partials, cudaStream_t st) {
-    if (total_tiles <= 0) return cudaSuccess;
-    momentum_kernel<<<total_tiles, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
+    if (total_groups <= 0) return cudaSuccess;
+    momentum_kernel<<<total_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
     return cudaGetLastError();
 }
 
@@ -349,10 +382,10 @@ cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partia
     return cudaGetLastError();
 }
 
-cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_tiles, const StepScalars& sc,
+cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_groups, const StepScalars& sc,
                                const float* s, int32_t xsel, int32_t use_s, cudaStream_t st) {
-    if (total_tiles <= 0) return cudaSuccess;
-    param_write_kernel<<<total_tiles, 256, 0, st>>>(d_mats, nmats, sc, s, xsel, use_s, device_status_ptr());
+    if (total_groups <= 0) return cudaSuccess;
+    param_write_kernel<<<total_groups, 256, 0, st>>>(d_mats, nmats, sc, s, xsel, use_s, device_status_ptr());
     return cudaGetLastError();
 }
 

@@ -321,36 +321,6 @@ __device__ __forceinline__ void epilogue_chunk_warp(const MatDev& md, int iter, 
     }
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
-}
-
-// L2 prefetch of a warp's block of a row-major matrix: rows [r0, r0 + nr) of
-// width `row_bytes` starting `col_byte0` bytes into each row, one 128-byte
-// line per lane per round.  Addresses stay inside the named rows.
-__device__ __forceinline__ void prefetch_block(const void* base, int64_t ld_bytes, int r0, int nr, int64_t col_byte0,
-                                               int64_t row_bytes, int lane) {
-    if (nr <= 0 || row_bytes <= 0) return;
-    const int lines = (int)((row_bytes + 127) / 128);
-    const char* b = static_cast<const char*>(base);
-    for (int i = lane; i < nr * lines; i += 32) {
-        const int rr = i / lines, ln = i - rr * lines;
-        prefetch_l2(b + (int64_t)(r0 + rr) * ld_bytes + col_byte0 + (int64_t)ln * 128);
-    }
-}
-
-// The fp32 master-X block the APPLY / FINAL epilogue of a tile reads, fetched
-// into L2 while the warp still waits for the accumulator.
-template <int ph>
-__device__ __forceinline__ void prefetch_tile_operands(const MatDev& md, int gi0, int gjb, int Mrows, int Ncols,
-                                                       int lane) {
-    if (ph != PH_APPLY && ph != PH_FINAL) return;
-    const int nr = min(32, Mrows - gi0);
-    const int nc = min(BN / 2, Ncols - gjb);
-    if (nr <= 0 || nc <= 0) return;
-    prefetch_block(md.xf[0], md.ldx * 4, gi0, nr, (int64_t)gjb * 4, (int64_t)nc * 4, lane);
-}
-
 // APPLY / FINAL epilogue of one warp over its chunks [qa, qb) of a tile:
 //   X <- s ((a + d_B,i) X + E_B X) into the fp32 master, plus (APPLY) the bf16
 //   operand copy the next iteration's GEMMs read.
@@ -602,15 +572,6 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             const int Mrows = md.r;
             const int Ncols = gemm ? md.c : md.r;
             const int gi0 = td.tm * C::TILE_M + (int)rank * BM + quad * 32;
-            // fetch the operands of this tile (first one only) and of the next into L2
-            // while the accumulator is still being computed
-            if (t == cluster_id) prefetch_tile_operands<ph>(md, gi0, td.tn * BN + half * (BN / 2), Mrows, Ncols, lane);
-            if (t + nclusters < ntiles) {
-                const TileDev tn2 = tiles[t + nclusters];
-                const MatDev& m2 = mats[tn2.mat];
-                prefetch_tile_operands<ph>(m2, tn2.tm * C::TILE_M + (int)rank * BM + quad * 32,
-                                           tn2.tn * BN + half * (BN / 2), m2.r, gemm ? m2.c : m2.r, lane);
-            }
             bool ok = true;
             if (lane == 0) ok = wait_bounded(tfull0 + 8 * acc, acc_phase, abort_flag, status);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;

@@ -34,7 +34,7 @@ struct MatDev {
     int32_t      mom_tiles_n; // momentum tiles along cols
     int32_t      mom_vec;     // 1: 16-byte vector access is legal for this matrix
     float        shape_scale; // sqrt(max(1, rows/cols))
-    int32_t      pad_;
+    int32_t      mom_grp0;    // first tile group (kMomGroup tiles per block) of this matrix
 };
 
 // One output tile of a grouped GEMM phase.
@@ -70,7 +70,8 @@ struct StepScalars {
     int32_t bf16_mode;
 };
 
-constexpr int kMomTile = 64;   // momentum kernel tile: 64 x 64 elements of M
+constexpr int kMomTile = 64;   // momentum / parameter-write tile: 64 x 64 elements of M or W
+constexpr int kMomGroup = 4;   // tiles one block of those kernels processes
 
 // launch timing hooks (profile.cu): slot = prof_before(class, stream); launch; prof_after(slot, stream)
 int prof_before(int cls, cudaStream_t s);
@@ -80,12 +81,12 @@ void prof_after(int slot, cudaStream_t s);
 int32_t* device_status_ptr();   // device address of this device's status word (nullptr on error)
 
 // ---- launchers (return cudaError_t of the launch) ----
-cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_tiles,
+cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_groups,
                             const StepScalars& sc, float* partials, cudaStream_t st);
 cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partials,
                         float* s_out, float eps, cudaStream_t st);
 // W <- W (1 - lr wd) - lr * scale * (use_s ? s : 1) * X, X from the fp32 master xf[xsel]
-cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_tiles, const StepScalars& sc,
+cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_groups, const StepScalars& sc,
                                const float* s, int32_t xsel, int32_t use_s, cudaStream_t st);
 cudaError_t launch_gemm_simt(Phase ph, const MatDev* d_mats, int32_t nmats, const TileDev* d_tiles, int32_t ntiles,
                              int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st);
