@@ -175,6 +175,48 @@ int mfsdp_muon_workspace_size(const mfsdp_matrix* mats, int32_t n, const mfsdp_m
 int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- owner-segment exchange fused into the step -------------------------
+ * Passage: arxivlens summary page, Abstract (deterministic owner-segment
+ * collectives: the ordinary backward reduction lands the full gradient on
+ * the owner, and forward/backward materialise parameters from the owner);
+ * gist.science French summary, Methodologie section 2, "Collectifs P2P
+ * Segment-Proprietaire" (gradient reduction writes only into the owner's
+ * segment; materialisation moves only non-empty owner segments to the ranks
+ * that need them).  mfsdp_muon_step_p2p is mfsdp_muon_step with both exchanges
+ * done inside its kernels over plain device pointers, which may point into
+ * peer GPUs' memory (NVLink / NVSwitch, with peer access enabled by the
+ * caller or memory mapped through CUDA IPC):
+ *   G = grad_parts[0] + grad_parts[1] + ... + grad_parts[nparts-1]
+ *       (summed in that order in fp32 inside the momentum kernel; the
+ *        matrix's own `grad` field is ignored and may be NULL)
+ *   after the step, the updated parameter is also stored, bit for bit, to
+ *   every param_copies[d] (inside the parameter-write kernel).
+ */
+#define MFSDP_MAX_PARTS  64
+#define MFSDP_MAX_COPIES 64
+
+typedef struct {
+    const void* const* grad_parts;   /* host array of nparts device pointers, rows x cols of grad_dtype,
+                                        each aligned to its element size; read only */
+    void* const*       param_copies; /* host array of ncopies device pointers, rows x cols of param_dtype,
+                                        aligned like param; written; NULL when ncopies = 0 */
+    int32_t            nparts;       /* 1..MFSDP_MAX_PARTS */
+    int32_t            ncopies;      /* 0..MFSDP_MAX_COPIES */
+} mfsdp_owner_segments;
+
+/* Workspace for mfsdp_muon_step_p2p (the descriptor table also holds the part
+ * and copy pointers).  segs: host array of n records, one per matrix. */
+int mfsdp_muon_workspace_size_p2p(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                                  const mfsdp_muon_hparams* hp, size_t* bytes);
+
+/* The grouped step with the gradient reduction and the parameter
+ * materialisation fused in (see above).  Same workspace rules, results and
+ * errors as mfsdp_muon_step; the result does not depend on where the parts and
+ * copies live.  Memory that aliases another matrix's buffers, or parts and
+ * copies that overlap, are the caller's error (peer memory cannot be checked). */
+int mfsdp_muon_step_p2p(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                        const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Number of kernel launches one mfsdp_muon_step call with these arguments enqueues. */
 int mfsdp_muon_step_launches(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
                              int32_t* launches);
@@ -259,6 +301,15 @@ int mfsdp_profile_end(mfsdp_profile* out);
 /* Synchronise `stream` and read (then clear) the device status word of the
  * current device: MFSDP_OK or the first MFSDP_ERR_* a kernel recorded. */
 int mfsdp_get_device_status(void* stream, int32_t* status);
+
+/* Failure-detection self-test: launches one CTA whose only wait (the same
+ * bounded mbarrier wait the GEMM engine uses, on a barrier that nothing
+ * arrives on) gives up after limit_ns (1e3..1e10) and records
+ * MFSDP_ERR_TIMEOUT in the device status word; the kernel then returns
+ * normally and the context stays usable.  Read the result with
+ * mfsdp_get_device_status().  Errors: MFSDP_ERR_INVALID_ARG, MFSDP_ERR_CUDA,
+ * MFSDP_ERR_UNSUPPORTED_DEVICE. */
+int mfsdp_selftest_bounded_wait(int64_t limit_ns, void* stream);
 
 /* Static text for a status code (never NULL). */
 const char* mfsdp_status_string(int32_t status);

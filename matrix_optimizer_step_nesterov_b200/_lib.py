@@ -38,7 +38,11 @@ EXPORTED = (
     "mfsdp_muon_step_launches", "mfsdp_muon_forget_workspace", "mfsdp_adamw_tail",
     "mfsdp_get_device_status", "mfsdp_status_string", "mfsdp_version",
     "mfsdp_profile_begin", "mfsdp_profile_end", "mfsdp_muon_step_noalloc",
+    "mfsdp_muon_workspace_size_p2p", "mfsdp_muon_step_p2p", "mfsdp_selftest_bounded_wait",
 )
+
+MFSDP_MAX_PARTS = 64
+MFSDP_MAX_COPIES = 64
 
 KCLASS_NAMES = ("momentum", "norm", "gram", "poly", "apply", "write", "adamw", "final")
 
@@ -78,6 +82,11 @@ class AdamWHParams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("reserved", ctypes.c_int32),
                 ("step", ctypes.c_int64)]
+
+
+class OwnerSegments(ctypes.Structure):
+    _fields_ = [("grad_parts", ctypes.POINTER(ctypes.c_void_p)), ("param_copies", ctypes.POINTER(ctypes.c_void_p)),
+                ("nparts", ctypes.c_int32), ("ncopies", ctypes.c_int32)]
 
 
 class Profile(ctypes.Structure):
@@ -124,8 +133,16 @@ def load() -> ctypes.CDLL:
     lib.mfsdp_profile_begin.restype = ctypes.c_int
     lib.mfsdp_profile_end.argtypes = [ctypes.POINTER(Profile)]
     lib.mfsdp_profile_end.restype = ctypes.c_int
+    lib.mfsdp_muon_workspace_size_p2p.argtypes = [ctypes.POINTER(Matrix), ctypes.POINTER(OwnerSegments), i32,
+                                                  ctypes.POINTER(MuonHParams), ctypes.POINTER(ctypes.c_size_t)]
+    lib.mfsdp_muon_workspace_size_p2p.restype = ctypes.c_int
+    lib.mfsdp_muon_step_p2p.argtypes = [ctypes.POINTER(Matrix), ctypes.POINTER(OwnerSegments), i32,
+                                        ctypes.POINTER(MuonHParams), p, ctypes.c_size_t, p]
+    lib.mfsdp_muon_step_p2p.restype = ctypes.c_int
     lib.mfsdp_muon_step_noalloc.argtypes = [ctypes.POINTER(Matrix), i32, ctypes.POINTER(MuonHParams), p]
     lib.mfsdp_muon_step_noalloc.restype = ctypes.c_int
+    lib.mfsdp_selftest_bounded_wait.argtypes = [i64, p]
+    lib.mfsdp_selftest_bounded_wait.restype = ctypes.c_int
     lib.mfsdp_version.argtypes = []
     lib.mfsdp_version.restype = ctypes.c_int32
     _lib = lib
@@ -225,6 +242,10 @@ def mfsdp_get_device_status(stream: int) -> int:
     return out.value
 
 
+def mfsdp_selftest_bounded_wait(limit_ns: int, stream: int) -> None:
+    _check(load().mfsdp_selftest_bounded_wait(int(limit_ns), stream), "mfsdp_selftest_bounded_wait")
+
+
 def mfsdp_version() -> int:
     return int(load().mfsdp_version())
 
@@ -254,3 +275,36 @@ def mfsdp_muon_step_noalloc(mats: Sequence[Matrix], hp: MuonHParams, stream: int
     Calls that overlap on the GPU share the scratch and race."""
     _check(load().mfsdp_muon_step_noalloc(matrix_array(mats), len(mats), ctypes.byref(hp), stream),
            "mfsdp_muon_step_noalloc")
+
+
+# ---- owner-segment exchange fused into the step -----------------------------------------
+
+def owner_segments(parts_per_matrix: Sequence[Sequence[int]], copies_per_matrix: Sequence[Sequence[int]]):
+    """OwnerSegments array from per-matrix lists of device pointers.  Returns
+    (array, keepalive): the pointer arrays must outlive every call using them."""
+    n = len(parts_per_matrix)
+    arr = (OwnerSegments * max(n, 1))()
+    keep = []
+    for i, (parts, copies) in enumerate(zip(parts_per_matrix, copies_per_matrix)):
+        pa = (ctypes.c_void_p * max(len(parts), 1))(*parts)
+        ca = (ctypes.c_void_p * max(len(copies), 1))(*copies)
+        keep += [pa, ca]
+        arr[i] = OwnerSegments(ctypes.cast(pa, ctypes.POINTER(ctypes.c_void_p)),
+                               ctypes.cast(ca, ctypes.POINTER(ctypes.c_void_p)) if copies else None,
+                               len(parts), len(copies))
+    return arr, keep
+
+
+def mfsdp_muon_workspace_size_p2p(mats: Sequence[Matrix], segs, hp: MuonHParams) -> int:
+    out = ctypes.c_size_t()
+    _check(load().mfsdp_muon_workspace_size_p2p(matrix_array(mats), segs, len(mats), ctypes.byref(hp),
+                                                ctypes.byref(out)), "mfsdp_muon_workspace_size_p2p")
+    return out.value
+
+
+def mfsdp_muon_step_p2p(mats: Sequence[Matrix], segs, hp: MuonHParams, workspace_ptr: int, workspace_bytes: int,
+                        stream: int, arr=None) -> None:
+    if arr is None:
+        arr = matrix_array(mats)
+    _check(load().mfsdp_muon_step_p2p(arr, segs, len(mats), ctypes.byref(hp), workspace_ptr, workspace_bytes,
+                                      stream), "mfsdp_muon_step_p2p")

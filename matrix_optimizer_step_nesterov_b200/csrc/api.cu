@@ -58,22 +58,39 @@ int validate_hparams(const mfsdp_muon_hparams* hp) {
     return MFSDP_OK;
 }
 
-int validate_matrix(const mfsdp_matrix& m) {
+int validate_matrix(const mfsdp_matrix& m, const mfsdp_owner_segments* seg) {
     if (m.rows < 0 || m.cols < 0) return MFSDP_ERR_INVALID_ARG;
     if (m.rows > (1LL << 30) || m.cols > (1LL << 30)) return MFSDP_ERR_INVALID_ARG;
     if (m.param_dtype != MFSDP_DTYPE_F32 && m.param_dtype != MFSDP_DTYPE_BF16) return MFSDP_ERR_UNSUPPORTED_DTYPE;
     if (m.grad_dtype != MFSDP_DTYPE_F32 && m.grad_dtype != MFSDP_DTYPE_BF16) return MFSDP_ERR_UNSUPPORTED_DTYPE;
     if (m.rows == 0 || m.cols == 0) return MFSDP_OK;
-    if (!m.param || !m.grad || !m.momentum) return MFSDP_ERR_INVALID_ARG;
-    if (!aligned(m.param, m.param_dtype == MFSDP_DTYPE_BF16 ? 2 : 4)) return MFSDP_ERR_MISALIGNED;
-    if (!aligned(m.grad, m.grad_dtype == MFSDP_DTYPE_BF16 ? 2 : 4)) return MFSDP_ERR_MISALIGNED;
+    if (!m.param || !m.momentum) return MFSDP_ERR_INVALID_ARG;
+    const size_t pe = m.param_dtype == MFSDP_DTYPE_BF16 ? 2 : 4;
+    const size_t ge = m.grad_dtype == MFSDP_DTYPE_BF16 ? 2 : 4;
+    if (!aligned(m.param, pe)) return MFSDP_ERR_MISALIGNED;
+    if (seg) {
+        if (seg->nparts < 1 || seg->nparts > MFSDP_MAX_PARTS || !seg->grad_parts) return MFSDP_ERR_INVALID_ARG;
+        if (seg->ncopies < 0 || seg->ncopies > MFSDP_MAX_COPIES) return MFSDP_ERR_INVALID_ARG;
+        if (seg->ncopies > 0 && !seg->param_copies) return MFSDP_ERR_INVALID_ARG;
+        for (int32_t r = 0; r < seg->nparts; ++r) {
+            if (!seg->grad_parts[r]) return MFSDP_ERR_INVALID_ARG;
+            if (!aligned(seg->grad_parts[r], ge)) return MFSDP_ERR_MISALIGNED;
+        }
+        for (int32_t d = 0; d < seg->ncopies; ++d) {
+            if (!seg->param_copies[d]) return MFSDP_ERR_INVALID_ARG;
+            if (!aligned(seg->param_copies[d], pe)) return MFSDP_ERR_MISALIGNED;
+        }
+    } else {
+        if (!m.grad) return MFSDP_ERR_INVALID_ARG;
+        if (!aligned(m.grad, ge)) return MFSDP_ERR_MISALIGNED;
+    }
     if (!aligned(m.momentum, 4)) return MFSDP_ERR_MISALIGNED;
     if (m.update_out && !aligned(m.update_out, 4)) return MFSDP_ERR_MISALIGNED;
     return MFSDP_OK;
 }
 
 // [begin, end) byte ranges of every user buffer, to reject aliasing between matrices
-int check_no_alias(const mfsdp_matrix* mats, int32_t n) {
+int check_no_alias(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n) {
     struct Range { uintptr_t b, e; int32_t owner; bool writable; };
     std::vector<Range> rs;
     rs.reserve(static_cast<size_t>(n) * 4);
@@ -84,7 +101,8 @@ int check_no_alias(const mfsdp_matrix* mats, int32_t n) {
         const uintptr_t pe = m.param_dtype == MFSDP_DTYPE_BF16 ? 2 : 4;
         const uintptr_t ge = m.grad_dtype == MFSDP_DTYPE_BF16 ? 2 : 4;
         rs.push_back({reinterpret_cast<uintptr_t>(m.param), reinterpret_cast<uintptr_t>(m.param) + numel * pe, i, true});
-        rs.push_back({reinterpret_cast<uintptr_t>(m.grad), reinterpret_cast<uintptr_t>(m.grad) + numel * ge, i, false});
+        if (!segs)
+            rs.push_back({reinterpret_cast<uintptr_t>(m.grad), reinterpret_cast<uintptr_t>(m.grad) + numel * ge, i, false});
         rs.push_back({reinterpret_cast<uintptr_t>(m.momentum), reinterpret_cast<uintptr_t>(m.momentum) + numel * 4, i, true});
         if (m.update_out)
             rs.push_back({reinterpret_cast<uintptr_t>(m.update_out), reinterpret_cast<uintptr_t>(m.update_out) + numel * 4, i, true});
@@ -115,6 +133,8 @@ struct Layout {
     std::vector<TileDev> sym_tiles;    // PH_GRAM
     std::vector<TileDev> poly_tiles;   // PH_POLY
     std::vector<TileDev> gen_tiles;    // PH_APPLY / PH_FINAL
+    std::vector<uint64_t> ptrs;        // owner-segment part and copy pointers, per matrix
+    size_t off_ptrs = 0;
     int32_t mom_tiles = 0;
     int32_t mom_groups = 0;
     size_t off_mats = 0, off_maps = 0, off_sym = 0, off_poly = 0, off_gen = 0, off_partials = 0, off_s = 0;
@@ -143,15 +163,32 @@ void build_tiles(Layout& L, Engine eng) {
     L.poly_tiles = L.sym_tiles;
 }
 
-int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp, char* base, Layout& L) {
+int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32_t n,
+                 const mfsdp_muon_hparams* hp, char* base, Layout& L) {
     const bool bf16 = hp->mode == MFSDP_MODE_BF16;
     L.engine = pick_engine(hp);
     L.mats.clear();
+    L.ptrs.clear();
+    std::vector<size_t> ptr_first;     // index into L.ptrs of each live matrix's part pointers
     int32_t tile0 = 0, grp0 = 0;
     for (int32_t i = 0; i < n; ++i) {
         const mfsdp_matrix& u = in[i];
         if (u.rows == 0 || u.cols == 0) continue;
         MatDev m{};
+        bool vec_parts = true;
+        if (segs) {
+            const mfsdp_owner_segments& sg = segs[i];
+            m.nparts = sg.nparts;
+            m.ncopies = sg.ncopies;
+            ptr_first.push_back(L.ptrs.size());
+            for (int32_t r = 0; r < sg.nparts; ++r) {
+                L.ptrs.push_back(reinterpret_cast<uint64_t>(sg.grad_parts[r]));
+                vec_parts = vec_parts && aligned(sg.grad_parts[r], u.grad_dtype == MFSDP_DTYPE_BF16 ? 8 : 16);
+            }
+            for (int32_t d = 0; d < sg.ncopies; ++d) L.ptrs.push_back(reinterpret_cast<uint64_t>(sg.param_copies[d]));
+        } else {
+            ptr_first.push_back(L.ptrs.size());
+        }
         m.param = u.param;
         m.grad = u.grad;
         m.buf = u.momentum;
@@ -173,7 +210,7 @@ int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp
         m.mom_grp0 = grp0;
         grp0 += static_cast<int32_t>((tiles + kMomGroup - 1) / kMomGroup);
         m.mom_vec = (u.cols % 4 == 0) && aligned(u.momentum, 16) &&
-                    aligned(u.grad, u.grad_dtype == MFSDP_DTYPE_BF16 ? 8 : 16);
+                    (segs ? vec_parts : aligned(u.grad, u.grad_dtype == MFSDP_DTYPE_BF16 ? 8 : 16));
         m.shape_scale = static_cast<float>(std::sqrt(std::max(1.0, static_cast<double>(u.rows) / u.cols)));
         L.mats.push_back(m);
     }
@@ -183,6 +220,13 @@ int build_layout(const mfsdp_matrix* in, int32_t n, const mfsdp_muon_hparams* hp
     const size_t nm = L.mats.size();
     size_t off = 0;
     L.off_mats = off;      off = align_up(off + nm * sizeof(MatDev));
+    L.off_ptrs = off;      off = align_up(off + L.ptrs.size() * sizeof(uint64_t));
+    for (size_t k = 0; k < nm; ++k) {
+        MatDev& m = L.mats[k];
+        const uint64_t* first = reinterpret_cast<const uint64_t*>(base ? base + L.off_ptrs : nullptr) + ptr_first[k];
+        m.gparts = m.nparts ? reinterpret_cast<const void* const*>(first) : nullptr;
+        m.pcopies = m.ncopies ? reinterpret_cast<void* const*>(first + m.nparts) : nullptr;
+    }
     L.maps_bytes = L.engine == Engine::Tc ? tc_maps_bytes(nm) : 0;
     L.off_maps = off;      off = align_up(off + L.maps_bytes);
     L.off_sym = off;       off = align_up(off + L.sym_tiles.size() * sizeof(TileDev));
@@ -229,39 +273,55 @@ struct CacheEntry { int dev; std::vector<char> head; };
 std::mutex g_cache_mu;
 std::unordered_map<uintptr_t, CacheEntry> g_cache;
 
-int validate_all(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp) {
+int validate_all(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                 const mfsdp_muon_hparams* hp) {
     if (n < 0) return MFSDP_ERR_INVALID_ARG;
     int st = validate_hparams(hp);
     if (st) return st;
     if (n > 0 && !mats) return MFSDP_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n; ++i) {
-        st = validate_matrix(mats[i]);
+        st = validate_matrix(mats[i], segs ? &segs[i] : nullptr);
         if (st) return st;
     }
-    return check_no_alias(mats, n);
+    return check_no_alias(mats, segs, n);
+}
+
+int workspace_size_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                        const mfsdp_muon_hparams* hp, size_t* bytes) {
+    if (!bytes) return MFSDP_ERR_INVALID_ARG;
+    int st = validate_all(mats, segs, n, hp);
+    if (st) return st;
+    Layout L;
+    st = build_layout(mats, segs, n, hp, nullptr, L);
+    if (st) return st;
+    *bytes = L.mats.empty() ? 0 : L.total;
+    return MFSDP_OK;
 }
 
 }  // namespace
+
+int muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                   const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes, void* stream);
+
 }  // namespace mfsdp
 
 using namespace mfsdp;
 
 extern "C" int mfsdp_muon_workspace_size(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
                                          size_t* bytes) {
-    if (!bytes) return MFSDP_ERR_INVALID_ARG;
-    int st = validate_all(mats, n, hp);
-    if (st) return st;
-    Layout L;
-    st = build_layout(mats, n, hp, nullptr, L);
-    if (st) return st;
-    *bytes = L.mats.empty() ? 0 : L.total;
-    return MFSDP_OK;
+    return workspace_size_impl(mats, nullptr, n, hp, bytes);
+}
+
+extern "C" int mfsdp_muon_workspace_size_p2p(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                                             const mfsdp_muon_hparams* hp, size_t* bytes) {
+    if (n > 0 && !segs) return MFSDP_ERR_INVALID_ARG;
+    return workspace_size_impl(mats, segs, n, hp, bytes);
 }
 
 extern "C" int mfsdp_muon_step_launches(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
                                         int32_t* launches) {
     if (!launches) return MFSDP_ERR_INVALID_ARG;
-    int st = validate_all(mats, n, hp);
+    int st = validate_all(mats, nullptr, n, hp);
     if (st) return st;
     int32_t live = 0;
     for (int32_t i = 0; i < n; ++i) live += (mats[i].rows > 0 && mats[i].cols > 0);
@@ -277,7 +337,19 @@ extern "C" int mfsdp_muon_forget_workspace(void* workspace) {
 
 extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
                                void* workspace, size_t workspace_bytes, void* stream) {
-    int st = validate_all(mats, n, hp);
+    return muon_step_impl(mats, nullptr, n, hp, workspace, workspace_bytes, stream);
+}
+
+extern "C" int mfsdp_muon_step_p2p(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                                   const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+    if (n > 0 && !segs) return MFSDP_ERR_INVALID_ARG;
+    return muon_step_impl(mats, segs, n, hp, workspace, workspace_bytes, stream);
+}
+
+int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                          const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes, void* stream) {
+    int st = validate_all(mats, segs, n, hp);
     if (st) return st;
     int32_t live = 0;
     for (int32_t i = 0; i < n; ++i) live += (mats[i].rows > 0 && mats[i].cols > 0);
@@ -288,7 +360,7 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     if (!aligned(workspace, kAlign)) return MFSDP_ERR_MISALIGNED;
     Layout L;
     char* base = static_cast<char*>(workspace);
-    st = build_layout(mats, n, hp, base, L);
+    st = build_layout(mats, segs, n, hp, base, L);
     if (st) return st;
     if (workspace_bytes < L.total) return MFSDP_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -296,6 +368,8 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     // head bytes: descriptor table and tile tables
     std::vector<char> head(L.off_partials, 0);
     std::memcpy(head.data() + L.off_mats, L.mats.data(), L.mats.size() * sizeof(MatDev));
+    if (!L.ptrs.empty())
+        std::memcpy(head.data() + L.off_ptrs, L.ptrs.data(), L.ptrs.size() * sizeof(uint64_t));
     if (L.maps_bytes && !tc_encode_maps(L.mats, head.data() + L.off_maps)) return MFSDP_ERR_CUDA;
     if (!L.sym_tiles.empty())
         std::memcpy(head.data() + L.off_sym, L.sym_tiles.data(), L.sym_tiles.size() * sizeof(TileDev));
@@ -337,7 +411,7 @@ extern "C" int mfsdp_muon_step(const mfsdp_matrix* mats, int32_t n, const mfsdp_
     sc.bf16_mode = hp->mode == MFSDP_MODE_BF16;
 
     int slot = prof_before(MFSDP_KCLASS_MOMENTUM, s);
-    cudaError_t e = launch_momentum(d_mats, nm, L.mom_groups, sc, d_partials, s);
+    cudaError_t e = launch_momentum(d_mats, nm, L.mom_groups, sc, d_partials, segs != nullptr, s);
     prof_after(slot, s);
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     slot = prof_before(MFSDP_KCLASS_NORM, s);
@@ -403,6 +477,16 @@ extern "C" int mfsdp_adamw_tail(float* p, const float* g, float* m, float* v, in
     const cudaError_t e = launch_adamw(p, g, m, v, n, hp->lr, hp->beta1, hp->beta2, hp->eps, decay, bc1, bc2, s);
     prof_after(slot, s);
     return e == cudaSuccess ? MFSDP_OK : MFSDP_ERR_CUDA;
+}
+
+extern "C" int mfsdp_selftest_bounded_wait(int64_t limit_ns, void* stream) {
+    if (limit_ns < 1000 || limit_ns > 10000000000LL) return MFSDP_ERR_INVALID_ARG;
+    int st = check_device();
+    if (st) return st;
+    return launch_bounded_wait_selftest(static_cast<unsigned long long>(limit_ns), static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? MFSDP_OK
+               : MFSDP_ERR_CUDA;
 }
 
 extern "C" int mfsdp_get_device_status(void* stream, int32_t* status) {

@@ -72,6 +72,7 @@ __device__ __forceinline__ T block_sum(T v, T* smem) {
 // writes buf, the fp32 master X (M, or M^T when rows > cols) and, in bf16
 // mode, its bf16 operand copy; each tile's sum of M^2 goes to partials[tile].
 // ---------------------------------------------------------------------------
+template <bool PARTS>
 __global__ void __launch_bounds__(256, 4)
 momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
                 float* __restrict__ partials, int32_t* status) {
@@ -85,6 +86,8 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     // fields used inside the tile loop, read once (the loop's stores could otherwise force reloads)
     float* __restrict__ bufp = md.buf;
     const void* gradp = md.grad;
+    const void* const* parts = md.gparts;   // owner-segment contributions (nparts > 0)
+    const int nparts = md.nparts;
     const int mom_vec = md.mom_vec, tiles_n = md.mom_tiles_n, tile0 = md.mom_tile0, grp0 = md.mom_grp0;
     const int64_t ntiles = tiles_m * md.mom_tiles_n;
     if (grp < grp0) {  // cannot happen with a host-built table
@@ -113,7 +116,16 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
             const int v = e * 256 + threadIdx.x;
             idx[e] = (i0 + (v >> 4)) * cols + j0 + (v & 15) * 4;
             b[e] = __ldcs(reinterpret_cast<const float4*>(bufp + idx[e]));
-            g[e] = load4(gradp, idx[e], gbf);
+            if (!PARTS) {
+                g[e] = load4(gradp, idx[e], gbf);
+            } else {
+                // the owner's gradient: contributions summed in rank order, in fp32
+                g[e] = load4(parts[0], idx[e], gbf);
+                for (int r = 1; r < nparts; ++r) {
+                    const float4 q = load4(parts[r], idx[e], gbf);
+                    g[e].x += q.x; g[e].y += q.y; g[e].z += q.z; g[e].w += q.w;
+                }
+            }
         }
         #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -148,7 +160,13 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
             const int64_t i = i0 + row, j = j0 + col;
             if (i < rows && j < cols) {
                 const int64_t idx = i * cols + j;
-                const float g = load_elem(gradp, idx, gbf);
+                float g;
+                if (!PARTS) {
+                    g = load_elem(gradp, idx, gbf);
+                } else {
+                    g = load_elem(parts[0], idx, gbf);
+                    for (int r = 1; r < nparts; ++r) g += load_elem(parts[r], idx, gbf);
+                }
                 const float b = beta * bufp[idx] + omb * g;
                 const float m = sc.nesterov ? (omb * g + beta * b) : b;
                 bufp[idx] = b;
@@ -239,8 +257,12 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
     float* wf = static_cast<float*>(md.param);
     __nv_bfloat16* wb = static_cast<__nv_bfloat16*>(md.param);
     float* uo = md.update_out;
-    const bool aligned_w = (cols % 4 == 0) && (reinterpret_cast<uintptr_t>(md.param) % (wbf ? 8 : 16) == 0) &&
-                           (uo == nullptr || reinterpret_cast<uintptr_t>(uo) % 16 == 0);
+    void* const* copies = md.pcopies;        // owner-segment destinations of the new parameter
+    const int ncopies = md.ncopies;
+    bool aligned_w = (cols % 4 == 0) && (reinterpret_cast<uintptr_t>(md.param) % (wbf ? 8 : 16) == 0) &&
+                     (uo == nullptr || reinterpret_cast<uintptr_t>(uo) % 16 == 0);
+    for (int d = 0; d < ncopies; ++d)
+        aligned_w = aligned_w && (reinterpret_cast<uintptr_t>(copies[d]) % (wbf ? 8 : 16) == 0);
     for (int k = 0; k < kMomGroup; ++k) {
     const int local = (grp - grp0) * kMomGroup + k;
     if (local >= ntiles) break;      // block-uniform
@@ -289,6 +311,10 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
             if (wbf) store4_bf16(wb, widx, w);
             else *reinterpret_cast<float4*>(wf + widx) = w;
             if (uo) *reinterpret_cast<float4*>(uo + widx) = o;
+            for (int d = 0; d < ncopies; ++d) {
+                if (wbf) store4_bf16(static_cast<__nv_bfloat16*>(copies[d]), widx, w);
+                else *reinterpret_cast<float4*>(static_cast<float*>(copies[d]) + widx) = w;
+            }
         }
     } else {
     for (int e = 0; e < 16; ++e) {
@@ -300,8 +326,15 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
         const float o = f * x;
         const int64_t idx = i * cols + j;
         if (uo) uo[idx] = o;
-        if (wbf) wb[idx] = __float2bfloat16_rn(fmaf(-lr, o, __bfloat162float(wb[idx]) * decay));
-        else wf[idx] = fmaf(-lr, o, wf[idx] * decay);
+        if (wbf) {
+            const __nv_bfloat16 nw = __float2bfloat16_rn(fmaf(-lr, o, __bfloat162float(wb[idx]) * decay));
+            wb[idx] = nw;
+            for (int d = 0; d < ncopies; ++d) static_cast<__nv_bfloat16*>(copies[d])[idx] = nw;
+        } else {
+            const float nw = fmaf(-lr, o, wf[idx] * decay);
+            wf[idx] = nw;
+            for (int d = 0; d < ncopies; ++d) static_cast<float*>(copies[d])[idx] = nw;
+        }
     }
     }
     __syncthreads();                 // tileX is reused by the next tile
@@ -323,23 +356,31 @@ __device__ __forceinline__ void adam_elem(float& p, float g, float& m, float& v,
     p = p * a.decay - a.lr * mhat / (sqrtf(vhat) + a.eps);
 }
 
+// Four 16-byte groups of each of p, g, m, v in flight per thread (16 loads)
+// before any arithmetic; streaming hints keep the one-pass tail from
+// displacing L2 contents.
 __global__ void __launch_bounds__(256)
 adamw_vec_kernel(float4* __restrict__ p, const float4* __restrict__ g, float4* __restrict__ m,
                  float4* __restrict__ v, int64_t n4, AdamScalars a) {
+    constexpr int U = 4;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += 2 * stride) {
-        const int64_t i2 = i + stride;
-        float4 P = p[i], G = __ldcs(g + i), M = m[i], V = v[i];
-        float4 P2, G2, M2, V2;
-        const bool two = i2 < n4;
-        if (two) { P2 = p[i2]; G2 = __ldcs(g + i2); M2 = m[i2]; V2 = v[i2]; }
-        adam_elem(P.x, G.x, M.x, V.x, a); adam_elem(P.y, G.y, M.y, V.y, a);
-        adam_elem(P.z, G.z, M.z, V.z, a); adam_elem(P.w, G.w, M.w, V.w, a);
-        p[i] = P; m[i] = M; v[i] = V;
-        if (two) {
-            adam_elem(P2.x, G2.x, M2.x, V2.x, a); adam_elem(P2.y, G2.y, M2.y, V2.y, a);
-            adam_elem(P2.z, G2.z, M2.z, V2.z, a); adam_elem(P2.w, G2.w, M2.w, V2.w, a);
-            p[i2] = P2; m[i2] = M2; v[i2] = V2;
+    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n4; i0 += U * stride) {
+        float4 P[U], G[U], M[U], V[U];
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < n4) {
+                P[u] = __ldcs(p + i); G[u] = __ldcs(g + i); M[u] = __ldcs(m + i); V[u] = __ldcs(v + i);
+            }
+        }
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < n4) {
+                adam_elem(P[u].x, G[u].x, M[u].x, V[u].x, a); adam_elem(P[u].y, G[u].y, M[u].y, V[u].y, a);
+                adam_elem(P[u].z, G[u].z, M[u].z, V[u].z, a); adam_elem(P[u].w, G[u].w, M[u].w, V[u].w, a);
+                __stcs(p + i, P[u]); __stcs(m + i, M[u]); __stcs(v + i, V[u]);
+            }
         }
     }
 }
@@ -369,9 +410,12 @@ int sm_count() {
 }  // namespace
 
 cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_groups,
-                            const StepScalars& sc, float* partials, cudaStream_t st) {
+                            const StepScalars& sc, float* partials, bool parts, cudaStream_t st) {
     if (total_groups <= 0) return cudaSuccess;
-    momentum_kernel<<<total_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
+    if (parts)
+        momentum_kernel<true><<<total_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
+    else
+        momentum_kernel<false><<<total_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
     return cudaGetLastError();
 }
 
@@ -398,8 +442,17 @@ cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, int64_t n
                      ((reinterpret_cast<uintptr_t>(p) | reinterpret_cast<uintptr_t>(g) |
                        reinterpret_cast<uintptr_t>(m) | reinterpret_cast<uintptr_t>(v)) % 16 == 0);
     const int64_t work = vec ? n / 4 : n;
-    int64_t blocks = (work + 2 * 256 - 1) / (2 * 256);
-    const int64_t cap = (int64_t)sm_count() * 8;
+    int64_t blocks = (work + 4 * 256 - 1) / (4 * 256);
+    // a grid of resident blocks only: the grid-stride loop then has no tail wave
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adamw_vec_kernel, 256, 0) != cudaSuccess ||
+            per_sm <= 0) {
+            cudaGetLastError();
+            per_sm = 2;
+        }
+    }
+    const int64_t cap = (int64_t)sm_count() * per_sm;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     if (vec) {

@@ -103,14 +103,14 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 // Bounded wait.  Returns false when the CTA is aborting (flag raised here on
 // timeout, or by another role).
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                             int32_t* status) {
+                                             int32_t* status, unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0u) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort_flag = 1;
                 if (status) atomicCAS(status, 0, -6 /* MFSDP_ERR_TIMEOUT */);
                 return false;
@@ -262,48 +262,54 @@ __device__ __forceinline__ void epilogue_chunk_warp(const MatDev& md, int iter, 
     if (ph == PH_GRAM || ph == PH_POLY) {
         // symmetric result: each element with row <= col is stored to both triangles
         __nv_bfloat16* ob = (ph == PH_GRAM) ? md.ab : static_cast<__nv_bfloat16*>(md.bm);
-        float ev[32];
         float di = 0.f, dj = 0.f;
         if (ph == PH_POLY) {
-            // E_A is symmetric: E[gi][gj] is read as E[gj][gi], consecutive across lanes
-            #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const int gj = gj0 + t;
-                ev[t] = (row_ok && gj < Ncols && gi < gj) ? md.af[(int64_t)gj * lda + gi] : 0.f;
-            }
             di = row_ok ? md.da[gi] : 0.f;
             dj = col_ok ? md.da[gjc] : 0.f;
         }
         const float s2 = sg * sg;
         #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int gj = gj0 + t;
-            const float acc = __uint_as_float(r[t]);
-            const float dt = (ph == PH_POLY) ? __shfl_sync(0xffffffffu, dj, t) : 0.f;   // d_A of column gj
-            float val = 0.f;
-            if (row_ok && gj < Ncols && gi <= gj) {
-                if (ph == PH_GRAM) {
-                    val = s2 * acc;
-                    if (gi == gj) {
-                        md.da[gi] = val;
-                        md.af[(int64_t)gi * lda + gi] = 0.f;
-                        ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
-                    } else {
-                        md.af[(int64_t)gj * lda + gi] = val;          // lower triangle, along column gj
-                        ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
-                    }
-                } else {
-                    if (gi == gj) {
-                        md.db[gi] = sc.b * di + sc.c * fmaf(di, di, acc);
-                        ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
-                    } else {
-                        const float e = ev[t];
-                        val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
-                        ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
-                    }
+        for (int h = 0; h < 32; h += 16) {           // two halves: 16 loads in flight, fewer registers
+            float ev[16];
+            if (ph == PH_POLY) {
+                // E_A is symmetric: E[gi][gj] is read as E[gj][gi], consecutive across lanes
+                #pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int gj = gj0 + h + k;
+                    ev[k] = (row_ok && gj < Ncols && gi < gj) ? md.af[(int64_t)gj * lda + gi] : 0.f;
                 }
             }
-            stg[lane][t] = val;
+            #pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int t = h + k;
+                const int gj = gj0 + t;
+                const float acc = __uint_as_float(r[t]);
+                const float dt = (ph == PH_POLY) ? __shfl_sync(0xffffffffu, dj, t) : 0.f;   // d_A of column gj
+                float val = 0.f;
+                if (row_ok && gj < Ncols && gi <= gj) {
+                    if (ph == PH_GRAM) {
+                        val = s2 * acc;
+                        if (gi == gj) {
+                            md.da[gi] = val;
+                            md.af[(int64_t)gi * lda + gi] = 0.f;
+                            ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
+                        } else {
+                            md.af[(int64_t)gj * lda + gi] = val;          // lower triangle, along column gj
+                            ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
+                        }
+                    } else {
+                        if (gi == gj) {
+                            md.db[gi] = sc.b * di + sc.c * fmaf(di, di, acc);
+                            ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
+                        } else {
+                            const float e = ev[k];
+                            val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
+                            ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
+                        }
+                    }
+                }
+                stg[lane][t] = val;
+            }
         }
         __syncwarp();
         // column domain: the upper-triangle copies (row gi0 + rr < column gjc)
@@ -622,6 +628,28 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
 }
 
 // ---------------------------------------------------------------------------
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// ever arrives on, with the engine's wait helper and a caller-given limit.  The
+// wait gives up, records MFSDP_ERR_TIMEOUT in the status word and the kernel
+// returns normally; the barrier is invalidated before the CTA exits.
+// ---------------------------------------------------------------------------
+__global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns, int32_t* status) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&bar), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        (void)wait_bounded(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
+        asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(&bar)) : "memory");
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -655,6 +683,11 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 }  // namespace
 
 bool tc_available() { return true; }
+
+cudaError_t launch_bounded_wait_selftest(unsigned long long limit_ns, cudaStream_t st) {
+    bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, device_status_ptr());
+    return cudaGetLastError();
+}
 
 size_t tc_maps_bytes(size_t nmats) { return nmats * sizeof(TcMaps); }
 

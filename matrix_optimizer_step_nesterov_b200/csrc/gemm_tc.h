@@ -22,6 +22,9 @@ bool tc_encode_maps(const std::vector<MatDev>& mats, void* host_out);
 void tc_build_tiles(const std::vector<MatDev>& mats, std::vector<TileDev>& gram, std::vector<TileDev>& poly,
                     std::vector<TileDev>& gen);
 
+// one CTA whose single wait runs out after limit_ns (failure-detection test)
+cudaError_t launch_bounded_wait_selftest(unsigned long long limit_ns, cudaStream_t st);
+
 cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, int32_t nmats,
                            const TileDev* d_tiles, int32_t ntiles, int32_t iter, const StepScalars& sc,
                            const float* s, cudaStream_t st);

@@ -35,6 +35,13 @@ struct MatDev {
     int32_t      mom_vec;     // 1: 16-byte vector access is legal for this matrix
     float        shape_scale; // sqrt(max(1, rows/cols))
     int32_t      mom_grp0;    // first tile group (kMomGroup tiles per block) of this matrix
+    // owner-segment exchange (mfsdp_muon_step_p2p): the gradient is the fixed-order
+    // sum of nparts contributions, and the updated parameter is also stored to
+    // ncopies destinations; device arrays of pointers in the workspace head
+    const void* const* gparts;
+    void* const*       pcopies;
+    int32_t      nparts;      // 0: the gradient is `grad`
+    int32_t      ncopies;
 };
 
 // One output tile of a grouped GEMM phase.
@@ -81,8 +88,9 @@ void prof_after(int slot, cudaStream_t s);
 int32_t* device_status_ptr();   // device address of this device's status word (nullptr on error)
 
 // ---- launchers (return cudaError_t of the launch) ----
+// parts: the gradients are owner-segment sums (MatDev::gparts) rather than MatDev::grad
 cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_groups,
-                            const StepScalars& sc, float* partials, cudaStream_t st);
+                            const StepScalars& sc, float* partials, bool parts, cudaStream_t st);
 cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partials,
                         float* s_out, float eps, cudaStream_t st);
 // W <- W (1 - lr wd) - lr * scale * (use_s ? s : 1) * X, X from the fp32 master xf[xsel]

@@ -42,23 +42,43 @@ class MuonOwnerStep:
     hold float32 tensors that receive the update O (tests), or None.
     """
 
-    def __init__(self, params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
+    def __init__(self, params: Sequence[torch.Tensor], grads: Sequence[Optional[torch.Tensor]],
                  momenta: Sequence[torch.Tensor], update_outs: Optional[Sequence[Optional[torch.Tensor]]] = None,
                  lr: float = 0.02, beta: float = 0.95, weight_decay: float = 0.01, eps: float = 1e-7,
                  a: float = 3.4445, b: float = -4.7750, c: float = 2.0315, ns_steps: int = 5,
-                 nesterov: bool = True, mode: str = "bf16"):
+                 nesterov: bool = True, mode: str = "bf16",
+                 grad_parts: Optional[Sequence[Sequence[torch.Tensor]]] = None,
+                 param_copies: Optional[Sequence[Sequence[torch.Tensor]]] = None):
+        """``grad_parts[i]`` (optional): the ranks' contributions to matrix i's
+        gradient, summed in order inside the step (``grads[i]`` may then be
+        None); ``param_copies[i]``: tensors that receive the updated parameter.
+        Either list turns the call into mfsdp_muon_step_p2p; the tensors may live
+        on peer GPUs that this device can access."""
         if not (len(params) == len(grads) == len(momenta)):
             raise ValueError("params, grads and momenta must have the same length")
         if update_outs is None:
             update_outs = [None] * len(params)
         self.mode = {"bf16": _lib.MFSDP_MODE_BF16, "fp32": _lib.MFSDP_MODE_FP32}[mode]
         self.hp = _lib.muon_hparams(lr, beta, weight_decay, eps, a, b, c, ns_steps, nesterov, self.mode)
+        p2p = grad_parts is not None or param_copies is not None
+        if p2p:
+            grad_parts = grad_parts if grad_parts is not None else [[g] for g in grads]
+            param_copies = param_copies if param_copies is not None else [[] for _ in params]
         mats: List[_lib.Matrix] = []
         for i, (w, g, m, o) in enumerate(zip(params, grads, momenta, update_outs)):
+            if p2p and g is None:
+                g = grad_parts[i][0]
             for t, nm in ((w, "param"), (g, "grad"), (m, "momentum")):
                 _check_tensor(t, f"{nm}[{i}]")
             if w.dim() != 2 or w.shape != g.shape or w.shape != m.shape:
                 raise ValueError(f"matrix {i}: param, grad and momentum must be 2D of equal shape")
+            if p2p:
+                for t in list(grad_parts[i]) + list(param_copies[i]):
+                    _check_tensor(t, f"segment tensor of matrix {i}")
+                    if t.shape != w.shape:
+                        raise ValueError(f"matrix {i}: grad parts and param copies must have the param's shape")
+                if any(t.dtype != g.dtype for t in grad_parts[i]) or any(t.dtype != w.dtype for t in param_copies[i]):
+                    raise TypeError(f"matrix {i}: parts take the grad dtype, copies the param dtype")
             if m.dtype != torch.float32:
                 raise TypeError(f"momentum[{i}] must be float32")
             if o is not None:
@@ -68,10 +88,17 @@ class MuonOwnerStep:
             mats.append(_lib.Matrix(w.data_ptr(), g.data_ptr(), m.data_ptr(),
                                     o.data_ptr() if o is not None else None,
                                     w.shape[0], w.shape[1], _dtype_code(w), _dtype_code(g)))
-        self._tensors = (list(params), list(grads), list(momenta), list(update_outs))
+        self._tensors = (list(params), list(grads), list(momenta), list(update_outs), grad_parts, param_copies)
         self.mats = mats
         self._arr = _lib.matrix_array(mats)
-        self.workspace_bytes = _lib.mfsdp_muon_workspace_size(mats, self.hp)
+        self._segs = None
+        if p2p:
+            self._segs, self._seg_keep = _lib.owner_segments(
+                [[t.data_ptr() for t in parts] for parts in grad_parts],
+                [[t.data_ptr() for t in copies] for copies in param_copies])
+            self.workspace_bytes = _lib.mfsdp_muon_workspace_size_p2p(mats, self._segs, self.hp)
+        else:
+            self.workspace_bytes = _lib.mfsdp_muon_workspace_size(mats, self.hp)
         dev = params[0].device if len(params) else torch.device("cuda")
         # 256-byte aligned workspace carved from a torch allocation
         self._ws = torch.empty(self.workspace_bytes + 256, dtype=torch.uint8, device=dev)
@@ -80,8 +107,12 @@ class MuonOwnerStep:
         self.launches = _lib.mfsdp_muon_step_launches(mats, self.hp)
 
     def step(self, stream: Optional[torch.cuda.Stream] = None) -> None:
-        _lib.mfsdp_muon_step(self.mats, self.hp, self.workspace_ptr, self.workspace_bytes,
-                             _stream_handle(stream), arr=self._arr)
+        if self._segs is not None:
+            _lib.mfsdp_muon_step_p2p(self.mats, self._segs, self.hp, self.workspace_ptr, self.workspace_bytes,
+                                     _stream_handle(stream), arr=self._arr)
+        else:
+            _lib.mfsdp_muon_step(self.mats, self.hp, self.workspace_ptr, self.workspace_bytes,
+                                 _stream_handle(stream), arr=self._arr)
 
     def close(self) -> None:
         if getattr(self, "_ws", None) is not None:

@@ -18,7 +18,7 @@ import torch
 
 import oracle
 from synth import workloads as W
-from synth.gen import matrix_inputs_many, tail_inputs
+from synth.gen import matrix_inputs_many, tail_inputs, round_to  # noqa: F401
 
 TOL_O = {"fp32": 1e-4, "bf16": 2e-2}
 TOL_BUF = 1e-6

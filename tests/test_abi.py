@@ -180,3 +180,26 @@ def test_adamw_validation(lib):
         lib.mfsdp_adamw_tail(0, 2 << 20, 3 << 20, 4 << 20, 16, hp, 0)
     assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
     lib.mfsdp_adamw_tail(0, 0, 0, 0, 0, hp, 0)   # n == 0 is a no-op
+
+
+def test_p2p_validation(lib):
+    hp = lib.muon_hparams()
+    m = lib.Matrix(1 << 20, 0, (1 << 20) + (1 << 24), None, 64, 64, 1, 1)   # grad NULL: parts carry it
+    segs, keep = lib.owner_segments([[1 << 26, 2 << 26]], [[3 << 26]])
+    assert lib.mfsdp_muon_workspace_size_p2p([m], segs, hp) > lib.mfsdp_muon_workspace_size(
+        [lib.Matrix(1 << 20, 1 << 25, (1 << 20) + (1 << 24), None, 64, 64, 1, 1)], hp) - 1
+    bad, keep2 = lib.owner_segments([[]], [[]])                      # no parts
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step_p2p([m], bad, hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    bad, keep3 = lib.owner_segments([[(1 << 26) + 1]], [[]])         # misaligned bf16 part
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step_p2p([m], bad, hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_MISALIGNED
+    bad, keep4 = lib.owner_segments([[1 << 26]], [[0]])              # NULL copy
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step_p2p([m], bad, hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    with pytest.raises(lib.MfsdpError) as e:                           # the plain entry point needs grad
+        lib.mfsdp_muon_step([m], hp, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG

@@ -72,7 +72,7 @@ def test_tiny_config_three_steps(mode):
 # ---- ragged shapes, edge cases -------------------------------------------------------
 
 RAGGED = [(1, 1), (1, 300), (300, 1), (100, 37), (37, 100), (129, 257), (257, 129), (65, 65),
-          (200, 1000), (1000, 200), (128, 128), (255, 513)]
+          (200, 1000), (1000, 200), (128, 128), (255, 513), (600, 1100), (1100, 600), (257, 2049)]
 
 
 @pytest.mark.parametrize("mode", MODES)
@@ -86,13 +86,16 @@ def test_ragged_shapes_grouped(mode, dtype):
         H.assert_parity(m, mode, f"{s.rows}x{s.cols}")
 
 
-@pytest.mark.parametrize("ns_steps", [0, 1, 3, 7])
-def test_iteration_counts(ns_steps):
-    wl = custom_workload([(96, 160), (160, 96)], dtype="f32", seed=5)
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("ns_steps", [0, 1, 2, 3, 7])
+def test_iteration_counts(ns_steps, mode):
+    # ns_steps = 1 makes the first iteration also the last (the Frobenius scale
+    # enters the final X update); 0 writes the normalised momentum itself
+    wl = custom_workload([(96, 160), (160, 96), (300, 520)], dtype="f32" if mode == "fp32" else "bf16", seed=5)
     hs = H.host_state(wl, wl.matrices)
-    res = H.gpu_step(hs, "fp32", ns_steps=ns_steps)
-    for k in range(2):
-        H.assert_parity(H.compare_matrix(hs, res, k, "fp32", ns_steps=ns_steps), "fp32")
+    res = H.gpu_step(hs, mode, ns_steps=ns_steps)
+    for k in range(3):
+        H.assert_parity(H.compare_matrix(hs, res, k, mode, ns_steps=ns_steps), mode)
 
 
 def test_plain_momentum_and_other_hparams():
