@@ -40,6 +40,7 @@ constexpr int NUM_EPI_WARPS = 8;                // two per TMEM lane quadrant, e
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int STG_BYTES = NUM_EPI_WARPS * 32 * 33 * 4;   // epilogue staging: one 32 x 33 fp32 buffer per epilogue warp
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr uint32_t kSuspendHintNs = 200000u;                // one suspended try_wait: at most ~0.2 ms
 
 // CTAs per MMA: 1 (cta_group::1, M = 128) or 2 (a cluster pair running
 // cta_group::2 MMAs of M = 256; each CTA loads its own 128 rows of A and half
@@ -94,6 +95,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test, but a thread whose phase is not complete yet is suspended
+// until it completes or about `hint_ns` nanoseconds pass, instead of
+// returning at once: a waiting thread issues nothing while it sleeps.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ unsigned long long globaltimer() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -106,15 +122,13 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
                                              int32_t* status, unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0u) {
-            if (*abort_flag) return false;
-            if (globaltimer() - t0 > limit_ns) {
-                *abort_flag = 1;
-                if (status) atomicCAS(status, 0, -6 /* MFSDP_ERR_TIMEOUT */);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > limit_ns) {
+            *abort_flag = 1;
+            if (status) atomicCAS(status, 0, -6 /* MFSDP_ERR_TIMEOUT */);
+            return false;
         }
     }
 }
