@@ -244,11 +244,12 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
             return p;
         };
         if (bf16) {
-            m.xf[0] = reinterpret_cast<float*>(take(x_elems * 4));
-            m.xf[1] = nullptr;
+            m.xf[0] = m.xf[1] = nullptr;
             m.xb[0] = reinterpret_cast<__nv_bfloat16*>(take(x_elems * 2));
             m.xb[1] = reinterpret_cast<__nv_bfloat16*>(take(x_elems * 2));
-            m.af = reinterpret_cast<float*>(take(a_elems * 4));
+            m.xlo[0] = reinterpret_cast<__nv_bfloat16*>(take(x_elems * 2));
+            m.xlo[1] = reinterpret_cast<__nv_bfloat16*>(take(x_elems * 2));
+            m.af = nullptr;
             m.ab = reinterpret_cast<__nv_bfloat16*>(take(a_elems * 2));
             m.bm = take(a_elems * 2);
             m.da = reinterpret_cast<float*>(take(static_cast<size_t>(m.r) * 4));
@@ -257,6 +258,7 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
             m.xf[0] = reinterpret_cast<float*>(take(x_elems * 4));
             m.xf[1] = reinterpret_cast<float*>(take(x_elems * 4));
             m.xb[0] = m.xb[1] = nullptr;
+            m.xlo[0] = m.xlo[1] = nullptr;
             m.af = reinterpret_cast<float*>(take(a_elems * 4));
             m.ab = nullptr;
             m.bm = take(a_elems * 4);
@@ -436,8 +438,9 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
             e = gemm(last ? PH_FINAL : PH_APPLY, d_gen, ngen, it, last ? MFSDP_KCLASS_FINAL : MFSDP_KCLASS_APPLY);
         if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     }
-    // the parameter write reads X from the fp32 master the last iteration wrote
-    const int32_t xsel = (hp->mode == MFSDP_MODE_BF16) ? 0 : (hp->ns_steps & 1);
+    // the parameter write reads X from the master copy the last iteration wrote
+    // (iteration it reads copy it & 1 and writes the other)
+    const int32_t xsel = hp->ns_steps & 1;
     slot = prof_before(MFSDP_KCLASS_WRITE, s);
     e = launch_param_write(d_mats, nm, L.mom_groups, sc, d_s, xsel, hp->ns_steps == 0 ? 1 : 0, s);
     prof_after(slot, s);

@@ -4,6 +4,7 @@
 // tail.  Method passages: arxivlens summary page of "MatrixFSDP", Abstract
 // (momentum-smoothed Muon update on the owner; tail on AdamW).
 #include "internal.h"
+#include "master.cuh"
 
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -41,6 +42,39 @@ __device__ __forceinline__ void store4_bf16(__nv_bfloat16* p, int64_t i, float4 
     *reinterpret_cast<uint2*>(p + i) = raw;
 }
 
+// bf16-mode master of X (master.cuh) at i..i+3, i % 4 == 0: hi and lo parts
+__device__ __forceinline__ void store4_master(__nv_bfloat16* xb, __nv_bfloat16* xlo, int64_t i, float4 v) {
+    uint16_t h0, h1, h2, h3, l0, l1, l2, l3;
+    master_split(v.x, h0, l0);
+    master_split(v.y, h1, l1);
+    master_split(v.z, h2, l2);
+    master_split(v.w, h3, l3);
+    *reinterpret_cast<uint2*>(xb + i) = make_uint2(static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16),
+                                                   static_cast<uint32_t>(h2) | (static_cast<uint32_t>(h3) << 16));
+    *reinterpret_cast<uint2*>(xlo + i) = make_uint2(static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16),
+                                                    static_cast<uint32_t>(l2) | (static_cast<uint32_t>(l3) << 16));
+}
+
+__device__ __forceinline__ void store1_master(__nv_bfloat16* xb, __nv_bfloat16* xlo, int64_t i, float v) {
+    uint16_t h, l;
+    master_split(v, h, l);
+    xb[i] = __ushort_as_bfloat16(h);
+    xlo[i] = __ushort_as_bfloat16(l);
+}
+
+__device__ __forceinline__ float4 load4_master(const __nv_bfloat16* xb, const __nv_bfloat16* xlo, int64_t i) {
+    const uint2 h = *reinterpret_cast<const uint2*>(xb + i);
+    const uint2 l = *reinterpret_cast<const uint2*>(xlo + i);
+    return make_float4(master_value(static_cast<uint16_t>(h.x & 0xFFFFu), static_cast<uint16_t>(l.x & 0xFFFFu)),
+                       master_value(static_cast<uint16_t>(h.x >> 16), static_cast<uint16_t>(l.x >> 16)),
+                       master_value(static_cast<uint16_t>(h.y & 0xFFFFu), static_cast<uint16_t>(l.y & 0xFFFFu)),
+                       master_value(static_cast<uint16_t>(h.y >> 16), static_cast<uint16_t>(l.y >> 16)));
+}
+
+__device__ __forceinline__ float load1_master(const __nv_bfloat16* xb, const __nv_bfloat16* xlo, int64_t i) {
+    return master_value(__bfloat16_as_ushort(xb[i]), __bfloat16_as_ushort(xlo[i]));
+}
+
 // index of the matrix owning tile group `grp` (largest i with mom_grp0 <= grp)
 __device__ __forceinline__ int find_matrix(const MatDev* mats, int nmats, int grp) {
     int lo = 0, hi = nmats - 1;
@@ -69,8 +103,9 @@ __device__ __forceinline__ T block_sum(T v, T* smem) {
 // ---------------------------------------------------------------------------
 // K1: one 64 x 64 tile of M per block of 256 threads.
 //   buf <- beta buf + (1-beta) G ;  M <- (1-beta) G + beta buf  (or M <- buf)
-// writes buf, the fp32 master X (M, or M^T when rows > cols) and, in bf16
-// mode, its bf16 operand copy; each tile's sum of M^2 goes to partials[tile].
+// writes buf and X = M, or M^T when rows > cols (bf16 mode: hi part, which is
+// the first GEMM operand, and remainder; fp32 mode: fp32); each tile's sum of
+// M^2 goes to partials[tile].
 // ---------------------------------------------------------------------------
 template <bool PARTS>
 __global__ void __launch_bounds__(256, 4)
@@ -102,8 +137,9 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
     const float beta = sc.beta, omb = 1.0f - sc.beta;
     const int tr = md.tr, gbf = md.grad_bf16, bf16_mode = sc.bf16_mode;
-    float* __restrict__ xf = md.xf[0];
-    __nv_bfloat16* __restrict__ xb = md.xb[0];
+    float* __restrict__ xf = md.xf[0];          // fp32 mode
+    __nv_bfloat16* __restrict__ xb = md.xb[0];  // bf16 mode: hi part ...
+    __nv_bfloat16* __restrict__ xl = md.xlo[0]; // ... and lo part
     const int64_t ldx = md.ldx;
     float sumsq = 0.f;
 
@@ -146,8 +182,8 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
             sumsq += m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
             if (!tr) {
                 const int64_t xi = (i0 + row) * ldx + j0 + col;
-                *reinterpret_cast<float4*>(xf + xi) = m;
-                if (bf16_mode) store4_bf16(xb, xi, m);
+                if (bf16_mode) store4_master(xb, xl, xi, m);
+                else *reinterpret_cast<float4*>(xf + xi) = m;
             } else {
                 tileM[row][col] = m.x; tileM[row][col + 1] = m.y;
                 tileM[row][col + 2] = m.z; tileM[row][col + 3] = m.w;
@@ -172,8 +208,8 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
                 bufp[idx] = b;
                 sumsq += m * m;
                 if (!tr) {
-                    xf[i * ldx + j] = m;
-                    if (bf16_mode) xb[i * ldx + j] = __float2bfloat16_rn(m);
+                    if (bf16_mode) store1_master(xb, xl, i * ldx + j, m);
+                    else xf[i * ldx + j] = m;
                 } else {
                     tileM[row][col] = m;
                 }
@@ -191,8 +227,8 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
                 const float4 m = make_float4(tileM[oc][orow], tileM[oc + 1][orow], tileM[oc + 2][orow],
                                              tileM[oc + 3][orow]);
                 const int64_t xi = (j0 + orow) * ldx + i0 + oc;
-                *reinterpret_cast<float4*>(xf + xi) = m;
-                if (bf16_mode) store4_bf16(xb, xi, m);
+                if (bf16_mode) store4_master(xb, xl, xi, m);
+                else *reinterpret_cast<float4*>(xf + xi) = m;
             }
         } else {
             for (int e = 0; e < 16; ++e) {
@@ -201,8 +237,8 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
                 const int64_t xr = j0 + orow, xc = i0 + ocol;
                 if (xr < cols && xc < rows) {
                     const float m = tileM[ocol][orow];
-                    xf[xr * ldx + xc] = m;
-                    if (bf16_mode) xb[xr * ldx + xc] = __float2bfloat16_rn(m);
+                    if (bf16_mode) store1_master(xb, xl, xr * ldx + xc, m);
+                    else xf[xr * ldx + xc] = m;
                 }
             }
         }
@@ -231,7 +267,8 @@ norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict_
 // Parameter write, one 64 x 64 tile of W per block (the momentum tiling):
 //   O = f * X (transposed back when rows > cols),  W <- W (1 - lr wd) - lr O
 // with f = shape scale, times s when no Newton-Schulz iteration ran (X is then
-// the unnormalised M).  X comes from the fp32 master buffer `xsel`.  A
+// the unnormalised M).  X comes from master copy `xsel` (hi part and remainder
+// in bf16 mode, fp32 in fp32 mode).  A
 // transposed X tile goes through shared memory so both X and W are read and
 // written along their rows; full tiles move 4 elements per access.
 __global__ void __launch_bounds__(256, 4)
@@ -251,7 +288,10 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
     const bool tr = md.tr != 0;
     const float f = md.shape_scale * (use_s ? s[mi] : 1.0f);
     const float lr = sc.lr, decay = sc.decay;
+    const bool bfm = sc.bf16_mode != 0;         // X as hi + remainder (bf16 mode) or fp32
     const float* __restrict__ xf = md.xf[xsel];
+    const __nv_bfloat16* __restrict__ xb = md.xb[xsel];
+    const __nv_bfloat16* __restrict__ xl = md.xlo[xsel];
     const int64_t ldx = md.ldx;
     const bool wbf = md.param_bf16 != 0;
     float* wf = static_cast<float*>(md.param);
@@ -263,12 +303,94 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
                      (uo == nullptr || reinterpret_cast<uintptr_t>(uo) % 16 == 0);
     for (int d = 0; d < ncopies; ++d)
         aligned_w = aligned_w && (reinterpret_cast<uintptr_t>(copies[d]) % (wbf ? 8 : 16) == 0);
+    // bf16 mode with a bf16 parameter: 8 elements per access (one 16-byte load
+    // each of X's hi part, X's lo part and W)
+    bool wide = bfm && wbf && (cols % 8 == 0) && (reinterpret_cast<uintptr_t>(md.param) % 16 == 0) &&
+                (uo == nullptr || reinterpret_cast<uintptr_t>(uo) % 16 == 0);
+    for (int d = 0; d < ncopies; ++d) wide = wide && (reinterpret_cast<uintptr_t>(copies[d]) % 16 == 0);
     for (int k = 0; k < kMomGroup; ++k) {
     const int local = (grp - grp0) * kMomGroup + k;
     if (local >= ntiles) break;      // block-uniform
     const int ti = local / tiles_n, tj = local % tiles_n;
     const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;   // W tile origin
     const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
+    if (full && wide) {
+        // thread: rows v >> 3 of the tile, 8 columns from (v & 7) * 8, for v = tid, tid + 256
+        float xv[2][8];
+        uint4 wv[2];
+        if (tr) {
+            #pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int v = e * 256 + threadIdx.x;
+                const int xr = v >> 3, xc = (v & 7) * 8;       // X tile row (a W column), 8 X columns (W rows)
+                const int64_t xi = (j0 + xr) * ldx + i0 + xc;
+                const uint4 h = __ldg(reinterpret_cast<const uint4*>(xb + xi));
+                const uint4 l = __ldg(reinterpret_cast<const uint4*>(xl + xi));
+                const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+                #pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    tileX[xr][xc + 2 * u] = master_value(static_cast<uint16_t>(hw[u] & 0xFFFFu),
+                                                         static_cast<uint16_t>(lw[u] & 0xFFFFu));
+                    tileX[xr][xc + 2 * u + 1] = master_value(static_cast<uint16_t>(hw[u] >> 16),
+                                                             static_cast<uint16_t>(lw[u] >> 16));
+                }
+            }
+        }
+        #pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            const int row = v >> 3, col = (v & 7) * 8;
+            wv[e] = *reinterpret_cast<const uint4*>(wb + (i0 + row) * cols + j0 + col);   // written below: no .nc
+            if (!tr) {
+                const int64_t xi = (i0 + row) * ldx + j0 + col;
+                const uint4 h = __ldg(reinterpret_cast<const uint4*>(xb + xi));
+                const uint4 l = __ldg(reinterpret_cast<const uint4*>(xl + xi));
+                const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+                #pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    xv[e][2 * u] = master_value(static_cast<uint16_t>(hw[u] & 0xFFFFu), static_cast<uint16_t>(lw[u] & 0xFFFFu));
+                    xv[e][2 * u + 1] = master_value(static_cast<uint16_t>(hw[u] >> 16), static_cast<uint16_t>(lw[u] >> 16));
+                }
+            }
+        }
+        if (tr) {
+            __syncthreads();
+            #pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int v = e * 256 + threadIdx.x;
+                const int row = v >> 3, col = (v & 7) * 8;
+                #pragma unroll
+                for (int u = 0; u < 8; ++u) xv[e][u] = tileX[col + u][row];
+            }
+        }
+        #pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int v = e * 256 + threadIdx.x;
+            const int row = v >> 3, col = (v & 7) * 8;
+            const int64_t widx = (i0 + row) * cols + j0 + col;
+            const uint32_t ww[4] = {wv[e].x, wv[e].y, wv[e].z, wv[e].w};
+            uint32_t nw[4];
+            float o[8];
+            #pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                o[2 * u] = f * xv[e][2 * u];
+                o[2 * u + 1] = f * xv[e][2 * u + 1];
+                const float w0 = __uint_as_float(ww[u] << 16), w1 = __uint_as_float(ww[u] & 0xFFFF0000u);
+                const __nv_bfloat162 n = __floats2bfloat162_rn(fmaf(-lr, o[2 * u], w0 * decay),
+                                                               fmaf(-lr, o[2 * u + 1], w1 * decay));
+                nw[u] = *reinterpret_cast<const uint32_t*>(&n);
+            }
+            const uint4 out = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+            *reinterpret_cast<uint4*>(wb + widx) = out;
+            if (uo) {
+                *reinterpret_cast<float4*>(uo + widx) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4*>(uo + widx + 4) = make_float4(o[4], o[5], o[6], o[7]);
+            }
+            for (int d = 0; d < ncopies; ++d) *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(copies[d]) + widx) = out;
+        }
+        __syncthreads();             // tileX is reused by the next tile
+        continue;
+    }
     if (tr) {
         // X tile rows = W columns j0.., X tile columns = W rows i0..
         if (full && (ldx % 4 == 0)) {
@@ -276,14 +398,18 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
             for (int e = 0; e < 4; ++e) {
                 const int v = e * 256 + threadIdx.x;
                 const int xr = v >> 4, xc = (v & 15) * 4;
-                const float4 x = *reinterpret_cast<const float4*>(xf + (j0 + xr) * ldx + i0 + xc);
+                const int64_t xi = (j0 + xr) * ldx + i0 + xc;
+                const float4 x = bfm ? load4_master(xb, xl, xi) : *reinterpret_cast<const float4*>(xf + xi);
                 tileX[xr][xc] = x.x; tileX[xr][xc + 1] = x.y; tileX[xr][xc + 2] = x.z; tileX[xr][xc + 3] = x.w;
             }
         } else {
             for (int e = 0; e < 16; ++e) {
                 const int v = e * 256 + threadIdx.x;
                 const int xr = v >> 6, xc = v & 63;
-                if (j0 + xr < cols && i0 + xc < rows) tileX[xr][xc] = xf[(j0 + xr) * ldx + i0 + xc];
+                if (j0 + xr < cols && i0 + xc < rows) {
+                    const int64_t xi = (j0 + xr) * ldx + i0 + xc;
+                    tileX[xr][xc] = bfm ? load1_master(xb, xl, xi) : xf[xi];
+                }
             }
         }
         __syncthreads();
@@ -296,6 +422,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
             const int v = e * 256 + threadIdx.x;
             const int row = v >> 4, col = (v & 15) * 4;
             if (tr) xv[e] = make_float4(tileX[col][row], tileX[col + 1][row], tileX[col + 2][row], tileX[col + 3][row]);
+            else if (bfm) xv[e] = load4_master(xb, xl, (i0 + row) * ldx + j0 + col);
             else xv[e] = *reinterpret_cast<const float4*>(xf + (i0 + row) * ldx + j0 + col);
             wv[e] = load4(md.param, (i0 + row) * cols + j0 + col, wbf);
         }
@@ -322,7 +449,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
         const int row = v >> 6, col = v & 63;
         const int64_t i = i0 + row, j = j0 + col;
         if (i >= rows || j >= cols) continue;
-        const float x = tr ? tileX[col][row] : xf[i * ldx + j];
+        const float x = tr ? tileX[col][row] : (bfm ? load1_master(xb, xl, i * ldx + j) : xf[i * ldx + j]);
         const float o = f * x;
         const int64_t idx = i * cols + j;
         if (uo) uo[idx] = o;

@@ -19,6 +19,7 @@
 // in their own waits, the producer drains the loads it has in flight, and
 // warp 1 frees TMEM before the CTA exits.
 #include "gemm_tc.h"
+#include "master.cuh"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -252,47 +253,67 @@ __host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major, int m) {
 }
 
 // ---------------------------------------------------------------------------
-// Warp-cooperative GRAM / POLY epilogue of one 32 x 32 chunk of the accumulator.
-// TMEM delivers it in the row domain: lane l holds row gi0 + l, columns
-// gj0 .. gj0 + 31.  Accesses that run along a column (the mirrored triangle
-// of a symmetric result, the transposed parameter write) are issued straight
-// from the row domain, where the 32 lanes touch 32 consecutive elements.
-// Accesses that run along a row go through the warp's 32 x 33 staging buffer
-// into the column domain (lane l takes column gj0 + l, rows one by one), so
-// they are coalesced too.
+// Epilogues.  Each epilogue warp owns 32 accumulator rows (its TMEM lane
+// quadrant) and 128 of the tile's 256 columns, in chunks of 32 x 32 read with
+// tcgen05.ld.  TMEM delivers a chunk in the row domain: lane l holds row
+// gi0 + l, columns gj0 .. gj0 + 31.  Accesses that run along a column (the
+// mirrored triangle of a symmetric result) are issued straight from the row
+// domain, where the 32 lanes touch 32 consecutive elements.  Accesses that run
+// along a row go through the warp's 32 x 33 staging buffer into the column
+// domain (lane l takes column gj0 + l, rows one by one), so they are coalesced
+// too.  Every global input is loaded one half chunk (16 rows or columns) ahead
+// of its use, and a tile's first half is loaded before the accumulator is
+// ready, while the MMAs still run.
 // ---------------------------------------------------------------------------
+
+// GRAM / POLY input of half chunk b of chunks [q0, ..): POLY reads E_A[gj][gi]
+// (E_A is symmetric; lanes address consecutive elements) for gj > gi.
 template <int ph>
-__device__ __forceinline__ void epilogue_chunk_warp(const MatDev& md, int iter, const StepScalars& sc,
-                                                    float sg, int gi0, int gj0, int Mrows, int Ncols,
-                                                    const uint32_t (&r)[32], float (*stg)[33], int lane) {
-    const int nxt = (iter & 1) ^ 1;
-    const int gi = gi0 + lane;      // row domain: this lane's row
-    const int gjc = gj0 + lane;     // column domain: this lane's column
-    const bool row_ok = gi < Mrows;
-    const bool col_ok = gjc < Ncols;
+__device__ __forceinline__ void sym_load_half(const MatDev& md, int gi, int gj_tile, int q0, int b, int Mrows,
+                                              int Ncols, int lane, unsigned short (&ev)[16], float& dj) {
+    if (ph != PH_POLY) return;
+    const unsigned short* ab = reinterpret_cast<const unsigned short*>(md.ab);
     const int64_t lda = md.lda;
-    // Every global load of a chunk is issued before any result is used, so the
-    // 32 loads of a lane are in flight together.
-    if (ph == PH_GRAM || ph == PH_POLY) {
-        // symmetric result: each element with row <= col is stored to both triangles
-        __nv_bfloat16* ob = (ph == PH_GRAM) ? md.ab : static_cast<__nv_bfloat16*>(md.bm);
-        float di = 0.f, dj = 0.f;
-        if (ph == PH_POLY) {
-            di = row_ok ? md.da[gi] : 0.f;
-            dj = col_ok ? md.da[gjc] : 0.f;
-        }
-        const float s2 = sg * sg;
+    const int gj0 = gj_tile + (q0 + (b >> 1)) * 32;
+    const int gjh = gj0 + (b & 1) * 16;
+    const bool row_ok = gi < Mrows;
+    #pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int gj = gjh + k;
+        ev[k] = (row_ok && gj < Ncols && gi < gj) ? __ldg(ab + (int64_t)gj * lda + gi) : (unsigned short)0;
+    }
+    if ((b & 1) == 0) dj = (gj0 + lane < Ncols) ? __ldg(md.da + gj0 + lane) : 0.f;   // d_A of column gj0 + lane
+}
+
+// GRAM / POLY epilogue of one warp over its live chunks [q0, q1):
+//   GRAM: A = s^2 acc  ->  E_A (bf16, both triangles), d_A
+//   POLY: B = b A + c A A with A A = acc + (d_i + d_j) E_A + d_i^2 delta_ij
+//         ->  E_B (bf16, both triangles), d_B
+// ev / dj hold the first half chunk's inputs, loaded by the caller.
+template <int ph>
+__device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepScalars& sc, float sg, int gi0,
+                                                  int gj_tile, int q0, int q1, int Mrows, int Ncols, uint32_t trow,
+                                                  float (*stg)[33], int lane, unsigned short (&ev)[16], float dj) {
+    const int gi = gi0 + lane;      // row domain: this lane's row
+    const bool row_ok = gi < Mrows;
+    const int64_t lda = md.lda;
+    __nv_bfloat16* ob = (ph == PH_GRAM) ? md.ab : static_cast<__nv_bfloat16*>(md.bm);
+    const float di = (ph == PH_POLY && row_ok) ? __ldg(md.da + gi) : 0.f;
+    const float s2 = sg * sg;
+    unsigned short en[16];
+    float djn = dj;
+    const int nb = 2 * (q1 - q0);
+    #pragma unroll 1
+    for (int q = q0; q < q1; ++q) {
+        const int gj0 = gj_tile + q * 32;
+        uint32_t r[32];
+        tmem_ld32(trow + q * 32, r);              // warp-collective
+        dj = djn;
         #pragma unroll
-        for (int h = 0; h < 32; h += 16) {           // two halves: 16 loads in flight, fewer registers
-            float ev[16];
-            if (ph == PH_POLY) {
-                // E_A is symmetric: E[gi][gj] is read as E[gj][gi], consecutive across lanes
-                #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int gj = gj0 + h + k;
-                    ev[k] = (row_ok && gj < Ncols && gi < gj) ? md.af[(int64_t)gj * lda + gi] : 0.f;
-                }
-            }
+        for (int hh = 0; hh < 2; ++hh) {          // the chunk's two halves (h known at compile time)
+            const int h = hh * 16;
+            const int b = 2 * (q - q0) + hh;
+            if (b + 1 < nb) sym_load_half<ph>(md, gi, gj_tile, q0, b + 1, Mrows, Ncols, lane, en, djn);
             #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int t = h + k;
@@ -305,18 +326,16 @@ __device__ __forceinline__ void epilogue_chunk_warp(const MatDev& md, int iter, 
                         val = s2 * acc;
                         if (gi == gj) {
                             md.da[gi] = val;
-                            md.af[(int64_t)gi * lda + gi] = 0.f;
                             ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
                         } else {
-                            md.af[(int64_t)gj * lda + gi] = val;          // lower triangle, along column gj
-                            ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
+                            ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);   // lower triangle, along column gj
                         }
                     } else {
                         if (gi == gj) {
                             md.db[gi] = sc.b * di + sc.c * fmaf(di, di, acc);
                             ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
                         } else {
-                            const float e = ev[k];
+                            const float e = bf16_bits_to_float(ev[k]);
                             val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
                             ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
                         }
@@ -324,55 +343,61 @@ __device__ __forceinline__ void epilogue_chunk_warp(const MatDev& md, int iter, 
                 }
                 stg[lane][t] = val;
             }
+            #pragma unroll
+            for (int k = 0; k < 16; ++k) ev[k] = en[k];
         }
         __syncwarp();
         // column domain: the upper-triangle copies (row gi0 + rr < column gjc)
+        const int gjc = gj0 + lane;
+        const bool col_ok = gjc < Ncols;
         #pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
             const int gi2 = gi0 + rr;
-            if (gi2 < Mrows && col_ok && gi2 < gjc) {
-                const float val = stg[rr][lane];
-                if (ph == PH_GRAM) md.af[(int64_t)gi2 * lda + gjc] = val;
-                ob[(int64_t)gi2 * lda + gjc] = __float2bfloat16_rn(val);
-            }
+            if (gi2 < Mrows && col_ok && gi2 < gjc) ob[(int64_t)gi2 * lda + gjc] = __float2bfloat16_rn(stg[rr][lane]);
         }
         __syncwarp();
-        return;
     }
 }
 
-// APPLY / FINAL epilogue of one warp over its chunks [qa, qb) of a tile:
-//   X <- s ((a + d_B,i) X + E_B X) into the fp32 master, plus (APPLY) the bf16
-//   operand copy the next iteration's GEMMs read.
-// X is read in the column domain (coalesced along its rows), 16 rows at a
-// time, and the loads of the next 16 rows are issued before the current ones
-// are computed and stored.
-template <int ph>
+// APPLY / FINAL input of half chunk b (16 rows of one 32-column chunk): the hi
+// and lo parts of X (master.cuh), copy `cur`, kept raw until used.
+__device__ __forceinline__ void x_load_half(const MatDev& md, int cur, int gi0, int gj_tile, int q0, int b,
+                                            int Mrows, int Ncols, int lane, unsigned short (&hv)[16],
+                                            unsigned short (&lv)[16]) {
+    const unsigned short* xh = reinterpret_cast<const unsigned short*>(md.xb[cur]);
+    const unsigned short* xlo = reinterpret_cast<const unsigned short*>(md.xlo[cur]);
+    const int gjc = gj_tile + (q0 + (b >> 1)) * 32 + lane;
+    const int h = (b & 1) * 16;
+    const bool ok = gjc < Ncols;
+    const int64_t base = (int64_t)(gi0 + h) * md.ldx + gjc;
+    #pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const bool in = ok && gi0 + h + k < Mrows;
+        hv[k] = in ? __ldg(xh + base + (int64_t)k * md.ldx) : (unsigned short)0;
+        lv[k] = in ? __ldg(xlo + base + (int64_t)k * md.ldx) : (unsigned short)0;
+    }
+}
+
+// APPLY / FINAL epilogue of one warp over its live chunks [q0, q1):
+//   X <- s ((a + d_B,i) X + E_B X)
+// X is read from copy iter & 1 (hi and lo parts, through the read-only path)
+// and written to the other copy; ch / cl hold the first half chunk, loaded by
+// the caller.
 __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, const StepScalars& sc, float sg,
-                                                int gi0, int gj_tile, int qa, int qb, int Mrows, int Ncols,
-                                                uint32_t trow, float (*stg)[33], int lane) {
-    float* xf = md.xf[0];
-    __nv_bfloat16* xbn = md.xb[(iter & 1) ^ 1];
+                                                int gi0, int gj_tile, int q0, int q1, int Mrows, int Ncols,
+                                                uint32_t trow, float (*stg)[33], int lane, unsigned short (&ch)[16],
+                                                unsigned short (&cl)[16]) {
+    const int cur = iter & 1;
+    unsigned short* __restrict__ xhn = reinterpret_cast<unsigned short*>(md.xb[cur ^ 1]);
+    unsigned short* __restrict__ xlon = reinterpret_cast<unsigned short*>(md.xlo[cur ^ 1]);
     const int64_t ldx = md.ldx;
     const int gi = gi0 + lane;
-    const float fa = gi < Mrows ? (sc.a + md.db[gi]) : 0.f;
-    int qe = qa;                                  // chunks [qa, qe) hold a column in range
-    while (qe < qb && gj_tile + qe * 32 < Ncols) ++qe;
-    const int nb = 2 * (qe - qa);                 // half-chunks of 16 rows
-    if (nb == 0) return;
-    auto load_half = [&](int b, float (&xv)[16]) {
-        const int gjc = gj_tile + (qa + (b >> 1)) * 32 + lane;
-        const int h = (b & 1) * 16;
-        const bool ok = gjc < Ncols;
-        const float* p = xf + (int64_t)(gi0 + h) * ldx + gjc;
-        #pragma unroll
-        for (int k = 0; k < 16; ++k) xv[k] = (ok && gi0 + h + k < Mrows) ? p[(int64_t)k * ldx] : 0.f;
-    };
-    float cur[16], nx[16];
-    load_half(0, cur);
+    const float fa = gi < Mrows ? (sc.a + __ldg(md.db + gi)) : 0.f;
+    unsigned short nh[16], nl[16];
+    const int nb = 2 * (q1 - q0);                 // half-chunks of 16 rows
     #pragma unroll 1
     for (int b = 0; b < nb; ++b) {
-        const int q = qa + (b >> 1);
+        const int q = q0 + (b >> 1);
         const int h = (b & 1) * 16;
         if (h == 0) {
             uint32_t r[32];
@@ -382,7 +407,7 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
             for (int t = 0; t < 32; ++t) stg[lane][t] = __uint_as_float(r[t]);
             __syncwarp();
         }
-        if (b + 1 < nb) load_half(b + 1, nx);
+        if (b + 1 < nb) x_load_half(md, cur, gi0, gj_tile, q0, b + 1, Mrows, Ncols, lane, nh, nl);
         float fk[16];                             // (a + d_B) of the 16 rows, gathered by every lane
         #pragma unroll
         for (int k = 0; k < 16; ++k) fk[k] = __shfl_sync(0xffffffffu, fa, h + k);
@@ -393,14 +418,19 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
                 const int rr = h + k;
                 if (gi0 + rr < Mrows) {
                     const int64_t idx = (int64_t)(gi0 + rr) * ldx + gjc;
-                    const float v = sg * fmaf(fk[k], cur[k], stg[rr][lane]);
-                    xf[idx] = v;
-                    if (ph == PH_APPLY) xbn[idx] = __float2bfloat16_rn(v);
+                    const float v = sg * fmaf(fk[k], master_value(ch[k], cl[k]), stg[rr][lane]);
+                    uint16_t hb, lb;
+                    master_split(v, hb, lb);
+                    xhn[idx] = hb;
+                    xlon[idx] = lb;
                 }
             }
         }
         #pragma unroll
-        for (int k = 0; k < 16; ++k) cur[k] = nx[k];
+        for (int k = 0; k < 16; ++k) {
+            ch[k] = nh[k];
+            cl[k] = nl[k];
+        }
     }
     __syncwarp();
 }
@@ -592,6 +622,25 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             const int Mrows = md.r;
             const int Ncols = gemm ? md.c : md.r;
             const int gi0 = td.tm * C::TILE_M + (int)rank * BM + quad * 32;
+            const int gj_tile = td.tn * BN;
+            // this warp's live chunks [q0, q1): columns in range and (symmetric
+            // phases) not entirely below the diagonal
+            int q0 = half * (BN / 64);
+            const int qb = q0 + BN / 64;
+            if (!gemm)
+                while (q0 < qb && gj_tile + q0 * 32 + 31 < gi0) ++q0;
+            int q1 = q0;
+            while (q1 < qb && gj_tile + q1 * 32 < Ncols) ++q1;
+            const bool live = gi0 < Mrows && q0 < q1;
+            // the first half chunk's inputs, loaded while the MMAs still run
+            unsigned short pre_a[16], pre_b[16];
+            float pre_dj = 0.f;
+            if (live) {
+                if constexpr (gemm)
+                    x_load_half(md, iter & 1, gi0, gj_tile, q0, 0, Mrows, Ncols, lane, pre_a, pre_b);
+                else
+                    sym_load_half<ph>(md, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, lane, pre_a, pre_dj);
+            }
             bool ok = true;
             if (lane == 0) ok = wait_bounded(tfull0 + 8 * acc, acc_phase, abort_flag, status);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -600,22 +649,13 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             const float sg = (iter == 0) ? s[td.mat] : 1.0f;
             const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
             float (*stg)[33] = reinterpret_cast<float (*)[33]>(stg_all + (warp - 2) * 32 * 33);
-            if constexpr (ph == PH_APPLY || ph == PH_FINAL) {
-                if (gi0 < Mrows)
-                    epilogue_x_warp<ph>(md, iter, sc, sg, gi0, td.tn * BN, half * (BN / 64), (half + 1) * (BN / 64),
-                                        Mrows, Ncols, trow, stg, lane);
-            } else {
-                #pragma unroll 1
-                for (int q = half * (BN / 64); q < (half + 1) * (BN / 64); ++q) {
-                    const int gj0 = td.tn * BN + q * 32;
-                    // warp-uniform skips: rows or columns out of range, or (symmetric
-                    // phases) a chunk entirely below the diagonal
-                    if (gi0 >= Mrows || gj0 >= Ncols) continue;
-                    if (!gemm && gj0 + 31 < gi0) continue;
-                    uint32_t r[32];
-                    tmem_ld32(trow + q * 32, r);       // warp-collective
-                    epilogue_chunk_warp<ph>(md, iter, sc, sg, gi0, gj0, Mrows, Ncols, r, stg, lane);
-                }
+            if (live) {
+                if constexpr (gemm)
+                    epilogue_x_warp(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_a,
+                                    pre_b);
+                else
+                    epilogue_sym_warp<ph>(md, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_a,
+                                          pre_dj);
             }
             tc_fence_before();
             __syncwarp();

@@ -16,10 +16,11 @@ struct MatDev {
     const void*  grad;        // G, rows x cols, grad dtype
     float*       buf;         // momentum, rows x cols fp32
     float*       update_out;  // optional O, rows x cols fp32
-    float*       xf[2];       // fp32 X: bf16 mode keeps one in-place master, fp32 mode ping-pongs
-    __nv_bfloat16* xb[2];     // bf16 X operands (bf16 mode), ping-pong
-    float*       af;          // fp32 E_A = A - diag(A), A = X X^T (r x r, zero diagonal)
-    __nv_bfloat16* ab;        // bf16 copy of E_A (bf16 mode GEMM operand)
+    float*       xf[2];       // fp32 mode: fp32 X, ping-pong (unused in bf16 mode)
+    __nv_bfloat16* xb[2];     // bf16 mode: hi part of X (the GEMM operand), ping-pong
+    __nv_bfloat16* xlo[2];    // bf16 mode: lo part of X (master.cuh), ping-pong with xb
+    float*       af;          // fp32 mode: E_A = A - diag(A), A = X X^T (r x r, zero diagonal)
+    __nv_bfloat16* ab;        // bf16 mode: E_A in bf16 (GEMM operand and epilogue input)
     void*        bm;          // E_B = B - diag(B), B = b A + c A A: bf16 (bf16 mode) or fp32
     float*       da;          // diag(A), r entries, fp32
     float*       db;          // diag(B), r entries, fp32
@@ -60,11 +61,11 @@ struct TileDev {
 // In bf16 mode this keeps the large diagonal terms (and the near-cancellation
 // a X + D_B X) out of bf16 rounding; the GEMM work is unchanged.
 enum Phase : int32_t {
-    PH_GRAM = 0,   // A = s^2 X X^T -> E_A (fp32 + operand copy), d_A   (upper tiles, mirrored)
+    PH_GRAM = 0,   // A = s^2 X X^T -> E_A, d_A                          (upper tiles, mirrored)
     PH_POLY = 1,   // B = b A + c A A -> E_B operand, d_B                (upper tiles, mirrored)
-    PH_APPLY = 2,  // X <- s ((a + d_B,i) X + E_B X)   (fp32 master + bf16 operand copy)
-    PH_FINAL = 3,  // last iteration: the same X update into the fp32 master only; the
-                   // parameter write then runs as its own HBM-bound kernel
+    PH_APPLY = 2,  // X <- s ((a + d_B,i) X + E_B X)
+    PH_FINAL = 3,  // the last iteration's X update (the same arithmetic); the parameter
+                   // write then runs as its own HBM-bound kernel
 };
 
 struct StepScalars {
@@ -93,7 +94,8 @@ cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_g
                             const StepScalars& sc, float* partials, bool parts, cudaStream_t st);
 cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partials,
                         float* s_out, float eps, cudaStream_t st);
-// W <- W (1 - lr wd) - lr * scale * (use_s ? s : 1) * X, X from the fp32 master xf[xsel]
+// W <- W (1 - lr wd) - lr * scale * (use_s ? s : 1) * X, X from master copy xsel
+// (bf16 mode: xb[xsel] + xlo[xsel]; fp32 mode: xf[xsel])
 cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_groups, const StepScalars& sc,
                                const float* s, int32_t xsel, int32_t use_s, cudaStream_t st);
 cudaError_t launch_gemm_simt(Phase ph, const MatDev* d_mats, int32_t nmats, const TileDev* d_tiles, int32_t ntiles,

@@ -167,7 +167,22 @@ def compare_matrix(hs: HostState, res: GpuResult, k: int, mode: str, **kw) -> Di
     return out
 
 
+def _report(metrics: Dict[str, float], mode: str, label: str) -> None:
+    """Append the measured errors to the JSON-lines file named by
+    MFSDP_PARITY_REPORT, when set (error margins for the design notes)."""
+    path = os.environ.get("MFSDP_PARITY_REPORT")
+    if not path:
+        return
+    import json
+    rec = {"label": label, "mode": mode}
+    rec.update({k: (float(v) if isinstance(v, (int, float, np.floating, np.integer)) else v)
+                for k, v in metrics.items()})
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
 def assert_parity(metrics: Dict[str, float], mode: str, label: str = "") -> None:
+    _report(metrics, mode, label)
     assert metrics["rel_O"] <= TOL_O[mode], f"{label} rel Frobenius error of O {metrics['rel_O']:.3e} > {TOL_O[mode]}"
     assert metrics["rel_buf"] <= TOL_BUF, f"{label} momentum rel error {metrics['rel_buf']:.3e}"
     if "write_excess" in metrics:

@@ -101,8 +101,8 @@ def test_workspace_size_is_host_only_and_grows_with_shapes(lib):
     s2 = lib.mfsdp_muon_workspace_size([_mat(lib, 512, 256)], hp)
     s3 = lib.mfsdp_muon_workspace_size([_mat(lib, 256, 1024)], hp)
     assert s1 == s2 > 0 and s3 > s1
-    # r x c = 256 x 512: fp32 master + two bf16 operands + fp32 A + bf16 A + bf16 B
-    assert s1 >= 256 * 512 * (4 + 2 + 2) + 256 * 256 * (4 + 2 + 2)
+    # r x c = 256 x 512: X as bf16 hi and lo parts, each ping-pong; bf16 E_A and E_B
+    assert s1 >= 256 * 512 * (2 + 2 + 2 + 2) + 256 * 256 * (2 + 2)
     hp32 = lib.muon_hparams(mode=lib.MFSDP_MODE_FP32)
     assert lib.mfsdp_muon_workspace_size([_mat(lib, 256, 512, pdt=0, gdt=0)], hp32) >= 256 * 512 * 8 + 256 * 256 * 8
     assert lib.mfsdp_muon_workspace_size([], hp) == 0

@@ -95,7 +95,8 @@ def test_iteration_counts(ns_steps, mode):
     hs = H.host_state(wl, wl.matrices)
     res = H.gpu_step(hs, mode, ns_steps=ns_steps)
     for k in range(3):
-        H.assert_parity(H.compare_matrix(hs, res, k, mode, ns_steps=ns_steps), mode)
+        H.assert_parity(H.compare_matrix(hs, res, k, mode, ns_steps=ns_steps), mode,
+                        f"ns_steps={ns_steps} {hs.specs[k].rows}x{hs.specs[k].cols}")
 
 
 def test_plain_momentum_and_other_hparams():
@@ -104,7 +105,7 @@ def test_plain_momentum_and_other_hparams():
     kw = dict(nesterov=False, lr=0.1, beta=0.9, weight_decay=0.1)
     res = H.gpu_step(hs, "fp32", **kw)
     for k in range(2):
-        H.assert_parity(H.compare_matrix(hs, res, k, "fp32", **kw), "fp32")
+        H.assert_parity(H.compare_matrix(hs, res, k, "fp32", **kw), "fp32", "plain momentum")
 
 
 @pytest.mark.parametrize("mode", MODES)
