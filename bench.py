@@ -474,7 +474,8 @@ def run_ours(args) -> int:
     mom = prof.get("momentum")
     mom_gbs = None
     if mom and mom[1] > 0:
-        mom_bytes = sum(s.numel for s in specs) * (16 if args.mode == "bf16" else 16)
+        # bf16 mode: G 2 + buf 4 in, buf 4 + X hi 2 + X lo 2 out; fp32 mode: G 4 + buf 4 in, buf 4 + X 4 out
+        mom_bytes = sum(s.numel for s in specs) * (14 if args.mode == "bf16" else 16)
         mom_gbs = round(mom_bytes * mom[0] / (mom[1] * 1e-3) / 1e9, 1)
 
     cpu_baseline = None

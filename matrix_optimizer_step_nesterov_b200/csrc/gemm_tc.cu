@@ -360,21 +360,25 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
 }
 
 // APPLY / FINAL input of half chunk b (16 rows of one 32-column chunk): the hi
-// and lo parts of X (master.cuh), copy `cur`, kept raw until used.
+// and lo parts of X (master.cuh), copy `cur`, kept raw until used.  Lane l
+// takes the column pair 2 (l & 15), 2 (l & 15) + 1 of rows of parity l >> 4,
+// so each access moves a bf16 pair and a warp covers two rows of 32 columns.
+// (A pair may reach one column past the matrix: into the padding of the
+// leading dimension, which nothing reads.)
 __device__ __forceinline__ void x_load_half(const MatDev& md, int cur, int gi0, int gj_tile, int q0, int b,
-                                            int Mrows, int Ncols, int lane, unsigned short (&hv)[16],
-                                            unsigned short (&lv)[16]) {
-    const unsigned short* xh = reinterpret_cast<const unsigned short*>(md.xb[cur]);
-    const unsigned short* xlo = reinterpret_cast<const unsigned short*>(md.xlo[cur]);
-    const int gjc = gj_tile + (q0 + (b >> 1)) * 32 + lane;
-    const int h = (b & 1) * 16;
+                                            int Mrows, int Ncols, int lane, uint32_t (&hv)[8], uint32_t (&lv)[8]) {
+    const uint32_t* xh = reinterpret_cast<const uint32_t*>(md.xb[cur]);
+    const uint32_t* xlo = reinterpret_cast<const uint32_t*>(md.xlo[cur]);
+    const int gjc = gj_tile + (q0 + (b >> 1)) * 32 + 2 * (lane & 15);
+    const int row0 = gi0 + (b & 1) * 16 + (lane >> 4);
     const bool ok = gjc < Ncols;
-    const int64_t base = (int64_t)(gi0 + h) * md.ldx + gjc;
+    const int64_t ldx = md.ldx;                    // even: a row is ldx / 2 pairs, two rows ldx pairs
+    const int64_t base = ((int64_t)row0 * ldx + gjc) >> 1;
     #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const bool in = ok && gi0 + h + k < Mrows;
-        hv[k] = in ? __ldg(xh + base + (int64_t)k * md.ldx) : (unsigned short)0;
-        lv[k] = in ? __ldg(xlo + base + (int64_t)k * md.ldx) : (unsigned short)0;
+    for (int k = 0; k < 8; ++k) {
+        const bool in = ok && row0 + 2 * k < Mrows;
+        hv[k] = in ? __ldg(xh + base + (int64_t)k * ldx) : 0u;
+        lv[k] = in ? __ldg(xlo + base + (int64_t)k * ldx) : 0u;
     }
 }
 
@@ -385,15 +389,16 @@ __device__ __forceinline__ void x_load_half(const MatDev& md, int cur, int gi0, 
 // the caller.
 __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, const StepScalars& sc, float sg,
                                                 int gi0, int gj_tile, int q0, int q1, int Mrows, int Ncols,
-                                                uint32_t trow, float (*stg)[33], int lane, unsigned short (&ch)[16],
-                                                unsigned short (&cl)[16]) {
+                                                uint32_t trow, float (*stg)[33], int lane, uint32_t (&ch)[8],
+                                                uint32_t (&cl)[8]) {
     const int cur = iter & 1;
-    unsigned short* __restrict__ xhn = reinterpret_cast<unsigned short*>(md.xb[cur ^ 1]);
-    unsigned short* __restrict__ xlon = reinterpret_cast<unsigned short*>(md.xlo[cur ^ 1]);
+    uint32_t* __restrict__ xhn = reinterpret_cast<uint32_t*>(md.xb[cur ^ 1]);
+    uint32_t* __restrict__ xlon = reinterpret_cast<uint32_t*>(md.xlo[cur ^ 1]);
     const int64_t ldx = md.ldx;
     const int gi = gi0 + lane;
-    const float fa = gi < Mrows ? (sc.a + __ldg(md.db + gi)) : 0.f;
-    unsigned short nh[16], nl[16];
+    const float fa = gi < Mrows ? (sc.a + __ldg(md.db + gi)) : 0.f;   // row domain: (a + d_B) of row gi
+    const int cp = lane & 15, rp = lane >> 4;
+    uint32_t nh[8], nl[8];
     const int nb = 2 * (q1 - q0);                 // half-chunks of 16 rows
     #pragma unroll 1
     for (int b = 0; b < nb; ++b) {
@@ -408,26 +413,26 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
             __syncwarp();
         }
         if (b + 1 < nb) x_load_half(md, cur, gi0, gj_tile, q0, b + 1, Mrows, Ncols, lane, nh, nl);
-        float fk[16];                             // (a + d_B) of the 16 rows, gathered by every lane
+        const int gjc = gj_tile + q * 32 + 2 * cp;
         #pragma unroll
-        for (int k = 0; k < 16; ++k) fk[k] = __shfl_sync(0xffffffffu, fa, h + k);
-        const int gjc = gj_tile + q * 32 + lane;
-        if (gjc < Ncols) {
-            #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int rr = h + k;
-                if (gi0 + rr < Mrows) {
-                    const int64_t idx = (int64_t)(gi0 + rr) * ldx + gjc;
-                    const float v = sg * fmaf(fk[k], master_value(ch[k], cl[k]), stg[rr][lane]);
-                    uint16_t hb, lb;
-                    master_split(v, hb, lb);
-                    xhn[idx] = hb;
-                    xlon[idx] = lb;
-                }
+        for (int k = 0; k < 8; ++k) {
+            const int rr = h + rp + 2 * k;        // row within the chunk
+            const float fk = __shfl_sync(0xffffffffu, fa, rr);
+            if (gjc < Ncols && gi0 + rr < Mrows) {
+                const float x0 = master_value(static_cast<uint16_t>(ch[k] & 0xFFFFu), static_cast<uint16_t>(cl[k] & 0xFFFFu));
+                const float x1 = master_value(static_cast<uint16_t>(ch[k] >> 16), static_cast<uint16_t>(cl[k] >> 16));
+                const float v0 = sg * fmaf(fk, x0, stg[rr][2 * cp]);
+                const float v1 = sg * fmaf(fk, x1, stg[rr][2 * cp + 1]);
+                uint16_t h0, l0, h1, l1;
+                master_split(v0, h0, l0);
+                master_split(v1, h1, l1);
+                const int64_t pidx = ((int64_t)(gi0 + rr) * ldx + gjc) >> 1;
+                xhn[pidx] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+                xlon[pidx] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
             }
         }
         #pragma unroll
-        for (int k = 0; k < 16; ++k) {
+        for (int k = 0; k < 8; ++k) {
             ch[k] = nh[k];
             cl[k] = nl[k];
         }
@@ -633,13 +638,14 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             while (q1 < qb && gj_tile + q1 * 32 < Ncols) ++q1;
             const bool live = gi0 < Mrows && q0 < q1;
             // the first half chunk's inputs, loaded while the MMAs still run
-            unsigned short pre_a[16], pre_b[16];
+            unsigned short pre_e[16];
+            uint32_t pre_h[8], pre_l[8];
             float pre_dj = 0.f;
             if (live) {
                 if constexpr (gemm)
-                    x_load_half(md, iter & 1, gi0, gj_tile, q0, 0, Mrows, Ncols, lane, pre_a, pre_b);
+                    x_load_half(md, iter & 1, gi0, gj_tile, q0, 0, Mrows, Ncols, lane, pre_h, pre_l);
                 else
-                    sym_load_half<ph>(md, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, lane, pre_a, pre_dj);
+                    sym_load_half<ph>(md, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, lane, pre_e, pre_dj);
             }
             bool ok = true;
             if (lane == 0) ok = wait_bounded(tfull0 + 8 * acc, acc_phase, abort_flag, status);
@@ -651,10 +657,10 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             float (*stg)[33] = reinterpret_cast<float (*)[33]>(stg_all + (warp - 2) * 32 * 33);
             if (live) {
                 if constexpr (gemm)
-                    epilogue_x_warp(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_a,
-                                    pre_b);
+                    epilogue_x_warp(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_h,
+                                    pre_l);
                 else
-                    epilogue_sym_warp<ph>(md, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_a,
+                    epilogue_sym_warp<ph>(md, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_e,
                                           pre_dj);
             }
             tc_fence_before();
