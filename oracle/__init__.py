@@ -38,4 +38,4 @@ from .muon import (  # noqa: F401
     muon_step,
 )
 from .adamw import AdamWHParams, adamw_step  # noqa: F401
-from .plan import plan_owners, PlanEntry, heaviest_rank  # noqa: F401
+from .plan import plan_owners, PlanEntry, heaviest_rank, reshard, ReshardRoute, state_bytes  # noqa: F401

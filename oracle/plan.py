@@ -31,6 +31,18 @@ Pins (tests/test_oracle_plan.py): every parameter owned exactly once; the
 result does not depend on the input order of equal items; brute-force optimal
 makespan on tiny instances within Graham's LPT bound; hand-checked balance of
 the Llama-shaped share plans.
+
+Owner-shard checkpoint resharding.  Source: the gist.science French and
+Portuguese summaries, Methodologie / Metodologia section 2, "Checkpointing et
+Routage" (checkpoints save the placement layout, the optimizer state is routed
+to the right owners through the MatrixShard metadata - Muon state for
+matrices, AdamW state for tails - and resharding works across world sizes).
+Reading taken here: a checkpoint holds each rank's owner-local buffers laid out
+by a saved plan; restoring on another world size plans the same parameters
+for the new world with the same rule, and every parameter's state is routed
+from (old owner, old offset) to (new owner, new offset).  The state that
+travels is the parameter and its fp32 momentum for a matrix, and fp32 p, m, v
+for a tail element.
 """
 
 from __future__ import annotations
@@ -137,3 +149,51 @@ def plan_owners(params: Sequence, world_size: int, steps: int = 5) -> Tuple[List
 
 def heaviest_rank(rank_flops: Sequence[float], rank_bytes: Sequence[int]) -> int:
     return min(range(len(rank_flops)), key=lambda r: (-rank_flops[r], -rank_bytes[r], r))
+
+
+@dataclasses.dataclass(frozen=True)
+class ReshardRoute:
+    pid: int
+    kind: int
+    src_rank: int
+    src_offset: int
+    dst_rank: int
+    dst_offset: int
+    elems: int
+    state_bytes: int
+
+
+def state_bytes(rows: int, cols: int, kind: int, dtype: str) -> int:
+    """Checkpointed state per parameter: the parameter and its fp32 momentum
+    (matrix) or fp32 p, m and v (tail element)."""
+    n = rows * cols
+    if kind == TAIL:
+        return 12 * n
+    return n * (_DTYPE_BYTES[dtype] + 4)
+
+
+def reshard(params: Sequence, old_entries: Sequence[PlanEntry], new_world: int,
+            steps: int = 5) -> Tuple[List[PlanEntry], List[ReshardRoute], int]:
+    """Plan ``params`` for ``new_world`` ranks and route every parameter's
+    state from its place in ``old_entries`` (a saved plan of the same
+    parameters, any world size) to its place in the new plan.
+
+    Returns (new entries, one route per parameter in input order, bytes of
+    state whose owner rank changes).
+    """
+    if len(old_entries) != len(params):
+        raise ValueError("the saved layout must describe the same parameters")
+    for p, e in zip(params, old_entries):
+        is_mat = p.kind == MATRIX
+        if e.pid != p.pid or e.rows != p.rows or e.cols != p.cols or e.kind != (MATRIX if is_mat else TAIL):
+            raise ValueError(f"saved record of parameter {p.pid} does not match its descriptor")
+    new_entries, _, _ = plan_owners(params, new_world, steps)
+    routes = []
+    for p, old, new in zip(params, old_entries, new_entries):
+        kind = MATRIX if p.kind == MATRIX else TAIL
+        routes.append(ReshardRoute(
+            pid=p.pid, kind=kind, src_rank=old.owner, src_offset=old.owner_offset,
+            dst_rank=new.owner, dst_offset=new.owner_offset, elems=p.rows * p.cols,
+            state_bytes=state_bytes(p.rows, p.cols, kind, p.dtype if kind == MATRIX else "f32")))
+    moved = sum(r.state_bytes for r in routes if r.src_rank != r.dst_rank)
+    return new_entries, routes, moved
