@@ -107,6 +107,49 @@ int mfsdp_plan(const mfsdp_param_desc* params, int64_t n, int32_t world_size, in
 int mfsdp_heaviest_rank(const double* rank_flops, const int64_t* rank_bytes, int32_t world_size,
                         int32_t* out_rank);
 
+/* ---- Owner-shard checkpoint resharding ----------------------------------
+ * Passage: gist.science French summary, Methodologie section 2, "Checkpointing
+ * et Routage" (and the Portuguese summary's Metodologia section 2): checkpoints
+ * save the placement layout, the optimizer state is routed to its owners
+ * through the MatrixShard metadata (Muon state for matrices, AdamW state for
+ * tails), and a checkpoint can be restored on another world size.
+ */
+
+/* Where one parameter's checkpointed state goes.  The state is the parameter
+ * and its fp32 momentum (matrix) or fp32 p, m, v (tail element); offsets are
+ * in elements of the owner's local buffer (matrices, parameter-id order) or of
+ * the packed tail, as in mfsdp_matrix_shard.owner_offset. */
+typedef struct {
+    int64_t param_id;
+    int32_t kind;            /* MFSDP_KIND_MATRIX or MFSDP_KIND_TAIL */
+    int32_t src_rank;        /* owner in the saved layout */
+    int32_t dst_rank;        /* owner in the new layout */
+    int32_t reserved;
+    int64_t src_offset;
+    int64_t dst_offset;
+    int64_t elems;           /* rows * cols */
+    int64_t state_bytes;     /* elems * (param bytes + 4) for a matrix, elems * 12 for a tail */
+} mfsdp_reshard_route;
+
+/*
+ * mfsdp_reshard - plan the parameters of a saved layout for another world size
+ * and route every parameter's state (host only, no CUDA call).
+ *   params           host array of n descriptors, those the saved layout was planned from
+ *   saved            host array of n MatrixShard records of the saved layout (any world size)
+ *   n                number of parameters, >= 0
+ *   new_world_size   >= 1
+ *   ns_steps         as for mfsdp_plan
+ *   out_shards       host array of n records, written: exactly mfsdp_plan(params, n, new_world_size, ns_steps)
+ *   out_routes       host array of n routes, written in input order
+ *   out_moved_bytes  state bytes of the parameters whose owner rank changes (may be NULL)
+ * Pure and deterministic.  Errors: MFSDP_ERR_INVALID_ARG (a NULL array with
+ * n > 0, a bad world size, a saved record whose id, shape or kind does not match
+ * its descriptor, or a negative saved owner or offset), and the errors of mfsdp_plan.
+ */
+int mfsdp_reshard(const mfsdp_param_desc* params, const mfsdp_matrix_shard* saved, int64_t n,
+                  int32_t new_world_size, int32_t ns_steps, mfsdp_matrix_shard* out_shards,
+                  mfsdp_reshard_route* out_routes, int64_t* out_moved_bytes);
+
 /* ---- Muon step --------------------------------------------------------
  * Passage: arxivlens summary page, Abstract (Muon orthogonalises
  * momentum-smoothed matrix updates with Newton-Schulz; the owner holds the

@@ -39,6 +39,7 @@ EXPORTED = (
     "mfsdp_get_device_status", "mfsdp_status_string", "mfsdp_version",
     "mfsdp_profile_begin", "mfsdp_profile_end", "mfsdp_muon_step_noalloc",
     "mfsdp_muon_workspace_size_p2p", "mfsdp_muon_step_p2p", "mfsdp_selftest_bounded_wait",
+    "mfsdp_reshard",
 )
 
 MFSDP_MAX_PARTS = 64
@@ -64,6 +65,12 @@ class MatrixShard(ctypes.Structure):
                 ("reserved", ctypes.c_int32), ("ns_flops", ctypes.c_double),
                 ("resident_bytes", ctypes.c_int64), ("owner_offset", ctypes.c_int64),
                 ("shape_scale", ctypes.c_double)]
+
+
+class ReshardRoute(ctypes.Structure):
+    _fields_ = [("param_id", ctypes.c_int64), ("kind", ctypes.c_int32), ("src_rank", ctypes.c_int32),
+                ("dst_rank", ctypes.c_int32), ("reserved", ctypes.c_int32), ("src_offset", ctypes.c_int64),
+                ("dst_offset", ctypes.c_int64), ("elems", ctypes.c_int64), ("state_bytes", ctypes.c_int64)]
 
 
 class Matrix(ctypes.Structure):
@@ -112,6 +119,10 @@ def load() -> ctypes.CDLL:
     lib.mfsdp_heaviest_rank.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), i32,
                                         ctypes.POINTER(ctypes.c_int32)]
     lib.mfsdp_heaviest_rank.restype = ctypes.c_int
+    lib.mfsdp_reshard.argtypes = [ctypes.POINTER(ParamDesc), ctypes.POINTER(MatrixShard), i64, i32, i32,
+                                  ctypes.POINTER(MatrixShard), ctypes.POINTER(ReshardRoute),
+                                  ctypes.POINTER(ctypes.c_int64)]
+    lib.mfsdp_reshard.restype = ctypes.c_int
     lib.mfsdp_muon_workspace_size.argtypes = [ctypes.POINTER(Matrix), i32, ctypes.POINTER(MuonHParams),
                                               ctypes.POINTER(ctypes.c_size_t)]
     lib.mfsdp_muon_workspace_size.restype = ctypes.c_int
@@ -182,6 +193,25 @@ def mfsdp_heaviest_rank(rank_flops: Sequence[float], rank_bytes: Sequence[int]) 
     out = ctypes.c_int32()
     _check(lib.mfsdp_heaviest_rank(f, b, R, ctypes.byref(out)), "mfsdp_heaviest_rank")
     return out.value
+
+
+def mfsdp_reshard(params: Sequence[tuple], saved: Sequence[MatrixShard], new_world_size: int, ns_steps: int = 5):
+    """params: (rows, cols, kind, dtype) per parameter; saved: its MatrixShard
+    records of the saved layout -> (new shards, routes, moved state bytes)."""
+    lib = load()
+    n = len(params)
+    arr = (ParamDesc * max(n, 1))()
+    for i, (r, c, k, d) in enumerate(params):
+        arr[i] = ParamDesc(int(r), int(c), int(k), int(d))
+    sv = (MatrixShard * max(n, 1))()
+    for i, rec in enumerate(saved):
+        sv[i] = rec
+    out = (MatrixShard * max(n, 1))()
+    routes = (ReshardRoute * max(n, 1))()
+    moved = ctypes.c_int64()
+    _check(lib.mfsdp_reshard(arr, sv, n, new_world_size, ns_steps, out, routes, ctypes.byref(moved)),
+           "mfsdp_reshard")
+    return list(out)[:n], list(routes)[:n], moved.value
 
 
 # ---- Muon step -----------------------------------------------------------------

@@ -152,3 +152,44 @@ extern "C" int mfsdp_heaviest_rank(const double* rank_flops, const int64_t* rank
     *out_rank = h;
     return MFSDP_OK;
 }
+
+// Owner-shard checkpoint resharding.  Passage: gist.science French summary,
+// Methodologie section 2, "Checkpointing et Routage" (saved placement layout,
+// optimizer state routed to its owners through the MatrixShard metadata,
+// restore across world sizes).  The new layout is the planner's own answer for
+// the new world size; each parameter's state goes from its saved (owner,
+// offset) to its new one.
+extern "C" int mfsdp_reshard(const mfsdp_param_desc* params, const mfsdp_matrix_shard* saved, int64_t n,
+                             int32_t new_world_size, int32_t ns_steps, mfsdp_matrix_shard* out_shards,
+                             mfsdp_reshard_route* out_routes, int64_t* out_moved_bytes) {
+    if (n < 0 || new_world_size < 1) return MFSDP_ERR_INVALID_ARG;
+    if (n > 0 && (!params || !saved || !out_shards || !out_routes)) return MFSDP_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < n; ++i) {
+        const mfsdp_param_desc& p = params[i];
+        const mfsdp_matrix_shard& s = saved[i];
+        const int32_t kind = p.kind == MFSDP_KIND_MATRIX ? MFSDP_KIND_MATRIX : MFSDP_KIND_TAIL;
+        if (s.param_id != i || s.rows != p.rows || s.cols != p.cols || s.kind != kind) return MFSDP_ERR_INVALID_ARG;
+        if (s.owner < 0 || s.owner_offset < 0) return MFSDP_ERR_INVALID_ARG;
+    }
+    const int st = mfsdp_plan(params, n, new_world_size, ns_steps, out_shards, nullptr, nullptr);
+    if (st != MFSDP_OK) return st;
+    int64_t moved = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        const mfsdp_param_desc& p = params[i];
+        const bool is_mat = p.kind == MFSDP_KIND_MATRIX;
+        const int64_t elems = p.rows * p.cols;
+        mfsdp_reshard_route& r = out_routes[i];
+        r.param_id = i;
+        r.kind = is_mat ? MFSDP_KIND_MATRIX : MFSDP_KIND_TAIL;
+        r.src_rank = saved[i].owner;
+        r.dst_rank = out_shards[i].owner;
+        r.reserved = 0;
+        r.src_offset = saved[i].owner_offset;
+        r.dst_offset = out_shards[i].owner_offset;
+        r.elems = elems;
+        r.state_bytes = is_mat ? elems * ((p.dtype == MFSDP_DTYPE_BF16 ? 2 : 4) + 4) : elems * 12;
+        if (r.src_rank != r.dst_rank) moved += r.state_bytes;
+    }
+    if (out_moved_bytes) *out_moved_bytes = moved;
+    return MFSDP_OK;
+}

@@ -203,3 +203,41 @@ def test_p2p_validation(lib):
     with pytest.raises(lib.MfsdpError) as e:                           # the plain entry point needs grad
         lib.mfsdp_muon_step([m], hp, 0, 0, 0)
     assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,old_w,new_w", [("7b_share", 8, 16), ("7b_share", 8, 5), ("32b_share", 64, 48),
+                                              ("block", 1, 4), ("skew", 4, 7), ("tiny", 1, 2)])
+def test_reshard_matches_oracle_exactly(lib, name, old_w, new_w):
+    wl = workload(name)
+    descs = _descs(wl)
+    saved, _, _ = lib.mfsdp_plan(descs, old_w)
+    shards, routes, moved = lib.mfsdp_reshard(descs, saved, new_w)
+    old_o, _, _ = oracle.plan_owners(wl.params, old_w)
+    new_o, routes_o, moved_o = oracle.reshard(wl.params, old_o, new_w)
+    assert [s.owner for s in shards] == [e.owner for e in new_o]
+    assert [s.owner_offset for s in shards] == [e.owner_offset for e in new_o]
+    assert [(r.param_id, r.kind, r.src_rank, r.src_offset, r.dst_rank, r.dst_offset, r.elems, r.state_bytes)
+            for r in routes] == [(o.pid, o.kind, o.src_rank, o.src_offset, o.dst_rank, o.dst_offset, o.elems,
+                                  o.state_bytes) for o in routes_o]
+    assert moved == moved_o
+    # the new layout is the planner's own answer for the new world size
+    direct, _, _ = lib.mfsdp_plan(descs, new_w)
+    assert [(s.owner, s.owner_offset) for s in direct] == [(s.owner, s.owner_offset) for s in shards]
+
+
+def test_reshard_validation(lib):
+    descs = [(64, 64, 0, 1), (32, 64, 0, 1)]
+    saved, _, _ = lib.mfsdp_plan(descs, 2)
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_reshard([(64, 64, 0, 1), (64, 32, 0, 1)], saved, 3)     # shape mismatch
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_reshard(descs, saved, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    bad = list(saved)
+    bad[1].owner = -1
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_reshard(descs, bad, 3)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    shards, routes, moved = lib.mfsdp_reshard([], [], 3)
+    assert shards == [] and routes == [] and moved == 0
