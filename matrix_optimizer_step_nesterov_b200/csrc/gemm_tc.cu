@@ -309,11 +309,35 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
         uint32_t r[32];
         tmem_ld32(trow + q * 32, r);              // warp-collective
         dj = djn;
+        // warp-uniform: the whole 32 x 32 chunk is inside the matrix and strictly above the diagonal
+        const bool interior = gi0 + 31 < Mrows && gj0 + 31 < Ncols && gi0 + 31 < gj0;
         #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {          // the chunk's two halves (h known at compile time)
             const int h = hh * 16;
             const int b = 2 * (q - q0) + hh;
             if (b + 1 < nb) sym_load_half<ph>(md, gi, gj_tile, q0, b + 1, Mrows, Ncols, lane, en, djn);
+            if (interior) {
+                // every element of the chunk lies strictly above the diagonal, inside the matrix
+                __nv_bfloat16* pm = ob + (int64_t)(gj0 + h) * lda + gi;   // E[gj][gi], gj = gj0 + h + k
+                #pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int t = h + k;
+                    const float acc = __uint_as_float(r[t]);
+                    float val;
+                    if (ph == PH_GRAM) {
+                        val = s2 * acc;
+                    } else {
+                        const float dt = __shfl_sync(0xffffffffu, dj, t);
+                        const float e = bf16_bits_to_float(ev[k]);
+                        val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
+                    }
+                    pm[(int64_t)k * lda] = __float2bfloat16_rn(val);
+                    stg[lane][t] = val;
+                }
+                #pragma unroll
+                for (int k = 0; k < 16; ++k) ev[k] = en[k];
+                continue;
+            }
             #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int t = h + k;
@@ -349,11 +373,18 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
         __syncwarp();
         // column domain: the upper-triangle copies (row gi0 + rr < column gjc)
         const int gjc = gj0 + lane;
-        const bool col_ok = gjc < Ncols;
-        #pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-            const int gi2 = gi0 + rr;
-            if (gi2 < Mrows && col_ok && gi2 < gjc) ob[(int64_t)gi2 * lda + gjc] = __float2bfloat16_rn(stg[rr][lane]);
+        if (interior) {
+            __nv_bfloat16* pu = ob + (int64_t)gi0 * lda + gjc;
+            #pragma unroll
+            for (int rr = 0; rr < 32; ++rr) pu[(int64_t)rr * lda] = __float2bfloat16_rn(stg[rr][lane]);
+        } else {
+            const bool col_ok = gjc < Ncols;
+            #pragma unroll
+            for (int rr = 0; rr < 32; ++rr) {
+                const int gi2 = gi0 + rr;
+                if (gi2 < Mrows && col_ok && gi2 < gjc)
+                    ob[(int64_t)gi2 * lda + gjc] = __float2bfloat16_rn(stg[rr][lane]);
+            }
         }
         __syncwarp();
     }
