@@ -405,6 +405,14 @@ __device__ __forceinline__ void x_load_half(const MatDev& md, int cur, int gi0, 
     const bool ok = gjc < Ncols;
     const int64_t ldx = md.ldx;                    // even: a row is ldx / 2 pairs, two rows ldx pairs
     const int64_t base = ((int64_t)row0 * ldx + gjc) >> 1;
+    if (gi0 + 32 <= Mrows && gj_tile + (q0 + (b >> 1)) * 32 + 32 <= Ncols) {   // warp-uniform: chunk inside X
+        #pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            hv[k] = __ldg(xh + base + (int64_t)k * ldx);
+            lv[k] = __ldg(xlo + base + (int64_t)k * ldx);
+        }
+        return;
+    }
     #pragma unroll
     for (int k = 0; k < 8; ++k) {
         const bool in = ok && row0 + 2 * k < Mrows;
@@ -445,11 +453,12 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
         }
         if (b + 1 < nb) x_load_half(md, cur, gi0, gj_tile, q0, b + 1, Mrows, Ncols, lane, nh, nl);
         const int gjc = gj_tile + q * 32 + 2 * cp;
+        const bool inside = gi0 + 32 <= Mrows && gj_tile + q * 32 + 32 <= Ncols;   // warp-uniform
         #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int rr = h + rp + 2 * k;        // row within the chunk
             const float fk = __shfl_sync(0xffffffffu, fa, rr);
-            if (gjc < Ncols && gi0 + rr < Mrows) {
+            if (inside || (gjc < Ncols && gi0 + rr < Mrows)) {
                 const float x0 = master_value(static_cast<uint16_t>(ch[k] & 0xFFFFu), static_cast<uint16_t>(cl[k] & 0xFFFFu));
                 const float x1 = master_value(static_cast<uint16_t>(ch[k] >> 16), static_cast<uint16_t>(cl[k] >> 16));
                 const float v0 = sg * fmaf(fk, x0, stg[rr][2 * cp]);
