@@ -75,6 +75,12 @@ def ns_flops_dense(specs, steps: int = 5) -> float:
     return tot
 
 
+# Per-launch DRAM bytes of the GEMM phases at the 7B share, from ncu on the
+# 4-matrix case: GRAM 0.594 GB x 6.54, POLY 0.249 GB x 7.0, APPLY 1.658 GB x 6.54,
+# averaged over 5 GRAM + 5 POLY + 5 APPLY/FINAL launches.
+GEMM_TRAFFIC_7B = round((5 * 0.594e9 * 6.54 + 5 * 0.249e9 * 7.0 + 5 * 1.658e9 * 6.54) / 15)
+
+
 def split_groups(specs, n_groups: int) -> List[List[int]]:
     """Matrix-index groups for the pipelined e2e measurement.  With three or
     more groups the first and the last hold a single small matrix, so that the
@@ -463,7 +469,12 @@ def run_ours(args) -> int:
         roof = {"bound": "tensor", "achieved": round(ns_tflops_kernel, 1) if ns_tflops_kernel else None,
                 "peak": peak, "unit": "TFLOP/s",
                 "frac": round(ns_tflops_kernel / peak, 4) if ns_tflops_kernel else None,
-                "traffic": None,
+                # ncu dram__bytes_read.sum + dram__bytes_write.sum of one GRAM, POLY and APPLY launch on
+                # 2 x 4096^2 + 4096x11008 + 11008x4096, scaled to the 7B share (GRAM and APPLY by X's
+                # elements, POLY by A's) and averaged over a step's 15 GEMM launches
+                "traffic": GEMM_TRAFFIC_7B if wl.name == "7b_share" else None,
+                "traffic_note": "scaled from a 4-matrix capture (profiles/tc_phase_kernel_4x4096.md)"
+                                if wl.name == "7b_share" else None,
                 "kernel": "Newton-Schulz GEMM phases (gram + poly + apply + final launches)",
                 "flops_per_launch": flops_alg * steps_timed / max(gemm_launches, 1),
                 "avg_launch_ms": gemm_ms / max(gemm_launches, 1),
