@@ -163,8 +163,10 @@ int mfsdp_reshard(const mfsdp_param_desc* params, const mfsdp_matrix_shard* save
  *   ns_steps times:  A = X X^T ;  B = b A + c A A ;  X <- a X + B X
  *   O = (transpose back) X * sqrt(max(1, rows/cols))
  *   W <- W (1 - lr wd) - lr O        (one round-to-nearest-even store to W's dtype)
- * MFSDP_MODE_BF16 rounds the GEMM operands (X, A, B) to bf16 and accumulates
- * in fp32; the master X, A in the b A term and every epilogue stay fp32.
+ * MFSDP_MODE_BF16 rounds the GEMM operands (X, A, B, without their diagonals)
+ * to bf16 and accumulates in fp32; the diagonals of A and B and all epilogue
+ * arithmetic stay fp32, and X is kept between iterations as bf16(X) plus
+ * bf16(X - bf16(X)), within 2^-16 of X.  MFSDP_MODE_FP32 is fp32 throughout.
  */
 typedef struct {
     void*       param;       /* device, rows x cols, param_dtype; updated in place */
