@@ -58,11 +58,16 @@ struct TcCfg {
 constexpr int kCtaGroup = 2;      // the engine's configuration
 
 // per-matrix TMA descriptors, stored in the workspace head (64-byte aligned)
+// E_A and E_B are stored block-upper: only the 256 x 256 tiles (I, J) with
+// I <= J are written, each in full.  An operand tile whose K block lies left of
+// the diagonal tile is read through the transposed (MN-major) view of tile (J, I).
 struct alignas(64) TcMaps {
     CUtensorMap xk[2];   // X bf16 operand, K-major view: dims {c, r}, box {64, 128}
     CUtensorMap xm[2];   // X bf16 operand, MN-major view: dims {c, r}, box {64, 64}
-    CUtensorMap ea;      // E_A bf16, dims {r, r}, box {64, 128}
-    CUtensorMap eb;      // E_B bf16, dims {r, r}, box {64, 128}
+    CUtensorMap ea;      // E_A bf16, K-major view: dims {r, r}, box {64, 128}
+    CUtensorMap eb;      // E_B bf16, K-major view: dims {r, r}, box {64, 128}
+    CUtensorMap eat;     // E_A bf16, MN-major view: dims {r, r}, box {64, 64}
+    CUtensorMap ebt;     // E_B bf16, MN-major view: dims {r, r}, box {64, 64}
 };
 
 // ---------------------------------------------------------------------------
@@ -242,11 +247,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
     return d;
 }
 
-// Instruction descriptor: D fp32, A/B bf16, A K-major, B K- or MN-major, N = 256, M = 128 or 256.
-__host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major, int m) {
+// Instruction descriptor: D fp32, A/B bf16, A and B K- or MN-major, N = 256, M = 128 or 256.
+__host__ __device__ constexpr uint32_t make_idesc(bool a_mn_major, bool b_mn_major, int m) {
     return (1u << 4)                 // D format: F32
          | (1u << 7)                 // A format: BF16
          | (1u << 10)                // B format: BF16
+         | ((a_mn_major ? 1u : 0u) << 15)
          | ((b_mn_major ? 1u : 0u) << 16)
          | (static_cast<uint32_t>(BN >> 3) << 17)
          | (static_cast<uint32_t>(m >> 4) << 24);
@@ -266,34 +272,61 @@ __host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major, int m) {
 // ready, while the MMAs still run.
 // ---------------------------------------------------------------------------
 
-// GRAM / POLY input of half chunk b of chunks [q0, ..): POLY reads E_A[gj][gi]
-// (E_A is symmetric; lanes address consecutive elements) for gj > gi.
+// GRAM / POLY input of half chunk b of chunks [q0, ..): POLY's E_A(gi, gj) for
+// the 16 columns gj of the half, gj > gi.
+//   off-diagonal tile: the tile's own elements E_A[gi][gj], 16 consecutive
+//     elements of this lane's row (two 16-byte loads);
+//   diagonal tile: the mirrored elements E_A[gj][gi], consecutive across lanes
+//     (the diagonal tile is stored with both triangles).
 template <int ph>
-__device__ __forceinline__ void sym_load_half(const MatDev& md, int gi, int gj_tile, int q0, int b, int Mrows,
-                                              int Ncols, int lane, unsigned short (&ev)[16], float& dj) {
+__device__ __forceinline__ void sym_load_half(const MatDev& md, bool offdiag, int gi, int gj_tile, int q0, int b,
+                                              int Mrows, int Ncols, int lane, unsigned short (&ev)[16], float& dj) {
     if (ph != PH_POLY) return;
     const unsigned short* ab = reinterpret_cast<const unsigned short*>(md.ab);
     const int64_t lda = md.lda;
     const int gj0 = gj_tile + (q0 + (b >> 1)) * 32;
     const int gjh = gj0 + (b & 1) * 16;
     const bool row_ok = gi < Mrows;
-    #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const int gj = gjh + k;
-        ev[k] = (row_ok && gj < Ncols && gi < gj) ? __ldg(ab + (int64_t)gj * lda + gi) : (unsigned short)0;
+    if (offdiag) {
+        if (row_ok && gjh + 16 <= Ncols) {
+            const uint4* p = reinterpret_cast<const uint4*>(ab + (int64_t)gi * lda + gjh);   // 16-byte aligned
+            const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
+            const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            #pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                ev[2 * k] = static_cast<unsigned short>(w[k] & 0xFFFFu);
+                ev[2 * k + 1] = static_cast<unsigned short>(w[k] >> 16);
+            }
+        } else {
+            #pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int gj = gjh + k;
+                ev[k] = (row_ok && gj < Ncols) ? __ldg(ab + (int64_t)gi * lda + gj) : (unsigned short)0;
+            }
+        }
+    } else {
+        #pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int gj = gjh + k;
+            ev[k] = (row_ok && gj < Ncols && gi < gj) ? __ldg(ab + (int64_t)gj * lda + gi) : (unsigned short)0;
+        }
     }
     if ((b & 1) == 0) dj = (gj0 + lane < Ncols) ? __ldg(md.da + gj0 + lane) : 0.f;   // d_A of column gj0 + lane
 }
 
 // GRAM / POLY epilogue of one warp over its live chunks [q0, q1):
-//   GRAM: A = s^2 acc  ->  E_A (bf16, both triangles), d_A
+//   GRAM: A = s^2 acc  ->  E_A (bf16), d_A
 //   POLY: B = b A + c A A with A A = acc + (d_i + d_j) E_A + d_i^2 delta_ij
-//         ->  E_B (bf16, both triangles), d_B
-// ev / dj hold the first half chunk's inputs, loaded by the caller.
+//         ->  E_B (bf16), d_B
+// Results are stored block-upper: an off-diagonal tile (I < J) writes only
+// itself; a diagonal tile writes its upper triangle and mirrors it into its
+// lower triangle.  ev / dj hold the first half chunk's inputs, loaded by the
+// caller.
 template <int ph>
-__device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepScalars& sc, float sg, int gi0,
-                                                  int gj_tile, int q0, int q1, int Mrows, int Ncols, uint32_t trow,
-                                                  float (*stg)[33], int lane, unsigned short (&ev)[16], float dj) {
+__device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepScalars& sc, float sg, bool offdiag,
+                                                  int gi0, int gj_tile, int q0, int q1, int Mrows, int Ncols,
+                                                  uint32_t trow, float (*stg)[33], int lane, unsigned short (&ev)[16],
+                                                  float dj) {
     const int gi = gi0 + lane;      // row domain: this lane's row
     const bool row_ok = gi < Mrows;
     const int64_t lda = md.lda;
@@ -315,7 +348,7 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
         for (int hh = 0; hh < 2; ++hh) {          // the chunk's two halves (h known at compile time)
             const int h = hh * 16;
             const int b = 2 * (q - q0) + hh;
-            if (b + 1 < nb) sym_load_half<ph>(md, gi, gj_tile, q0, b + 1, Mrows, Ncols, lane, en, djn);
+            if (b + 1 < nb) sym_load_half<ph>(md, offdiag, gi, gj_tile, q0, b + 1, Mrows, Ncols, lane, en, djn);
             if (interior) {
                 // every element of the chunk lies strictly above the diagonal, inside the matrix
                 __nv_bfloat16* pm = ob + (int64_t)(gj0 + h) * lda + gi;   // E[gj][gi], gj = gj0 + h + k
@@ -331,7 +364,7 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
                         const float e = bf16_bits_to_float(ev[k]);
                         val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
                     }
-                    pm[(int64_t)k * lda] = __float2bfloat16_rn(val);
+                    if (!offdiag) pm[(int64_t)k * lda] = __float2bfloat16_rn(val);   // mirror inside the diagonal tile
                     stg[lane][t] = val;
                 }
                 #pragma unroll
@@ -351,7 +384,7 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
                         if (gi == gj) {
                             md.da[gi] = val;
                             ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
-                        } else {
+                        } else if (!offdiag) {
                             ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);   // lower triangle, along column gj
                         }
                     } else {
@@ -361,7 +394,7 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
                         } else {
                             const float e = bf16_bits_to_float(ev[k]);
                             val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
-                            ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
+                            if (!offdiag) ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
                         }
                     }
                 }
@@ -483,6 +516,13 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
 // ---------------------------------------------------------------------------
 // the persistent kernel
 // ---------------------------------------------------------------------------
+// Which operands come from block-upper E storage: A of POLY, APPLY and FINAL
+// (E_A, E_B) and B of POLY (E_A).
+template <int ph>
+constexpr bool kSymA = ph == PH_POLY || ph == PH_APPLY || ph == PH_FINAL;
+template <int ph>
+constexpr bool kSymB = ph == PH_POLY;
+
 template <int ph, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps, int32_t nmats,
@@ -558,6 +598,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                 const int nk = (K + BK - 1) / BK;
                 const CUtensorMap* amap = (ph == PH_GRAM) ? &mp.xk[cur] : (ph == PH_POLY) ? &mp.ea : &mp.eb;
                 const CUtensorMap* bmap = (ph == PH_GRAM) ? &mp.xk[cur] : (ph == PH_POLY) ? &mp.ea : &mp.xm[cur];
+                const CUtensorMap* amap_t = (ph == PH_POLY) ? &mp.eat : &mp.ebt;   // A of POLY / APPLY
                 const int i0 = td.tm * C::TILE_M + (int)rank * BM;        // this CTA's A rows
                 const int jb = td.tn * BN + (int)rank * C::B_ROWS;        // this CTA's share of B
                 for (int kb = 0; kb < nk; ++kb) {
@@ -565,31 +606,31 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                     const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
                     const uint32_t sb = sa + A_BYTES;
                     const uint32_t fb = full0 + 8 * stage;
-                    if (CG == 1) {
-                        mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                        tma_load_2d(sa, amap, fb, kb * BK, i0);
-                        if (!gemm) {
-                            #pragma unroll
-                            for (int h = 0; h < C::B_ROWS / 128; ++h)
-                                tma_load_2d(sb + h * (128 * BK * 2), bmap, fb, kb * BK, jb + 128 * h);
-                        } else {
-                            #pragma unroll
-                            for (int q = 0; q < C::B_ROWS / 64; ++q)
-                                tma_load_2d(sb + q * (BK * 128), bmap, fb, jb + 64 * q, kb * BK);
-                        }
+                    // block-upper storage: K blocks left of the operand's own diagonal tile
+                    // come from the transposed tile
+                    const int kt = kb / (BN / BK);
+                    const bool a_t = kSymA<ph> && kt < td.tm;
+                    const bool b_t = kSymB<ph> && kt < td.tn;
+                    if (CG == 1) mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    else if (leader) mbar_arrive_expect_tx(fb, CG * STAGE_BYTES);   // both CTAs' bytes
+                    const uint32_t fbl = (CG == 2) ? map_to_rank(fb, 0) : fb;
+                    auto load = [&](uint32_t dst, const CUtensorMap* map, int x, int y) {
+                        if (CG == 2) tma_load_2d_pair(dst, map, fbl, x, y);
+                        else tma_load_2d(dst, map, fbl, x, y);
+                    };
+                    if (a_t) {
+                        load(sa, amap_t, i0, kb * BK);               // A rows i0 .. i0 + 63, MN-major
+                        load(sa + BK * 128, amap_t, i0 + 64, kb * BK);
                     } else {
-                        if (leader) mbar_arrive_expect_tx(fb, CG * STAGE_BYTES);   // both CTAs' bytes
-                        const uint32_t fbl = map_to_rank(fb, 0);
-                        tma_load_2d_pair(sa, amap, fbl, kb * BK, i0);
-                        if (!gemm) {
-                            #pragma unroll
-                            for (int h = 0; h < C::B_ROWS / 128; ++h)
-                                tma_load_2d_pair(sb + h * (128 * BK * 2), bmap, fbl, kb * BK, jb + 128 * h);
-                        } else {
-                            #pragma unroll
-                            for (int q = 0; q < C::B_ROWS / 64; ++q)
-                                tma_load_2d_pair(sb + q * (BK * 128), bmap, fbl, jb + 64 * q, kb * BK);
-                        }
+                        load(sa, amap, kb * BK, i0);
+                    }
+                    if (gemm || b_t) {
+                        const CUtensorMap* bm_ = gemm ? bmap : &mp.eat;
+                        #pragma unroll
+                        for (int q = 0; q < C::B_ROWS / 64; ++q) load(sb + q * (BK * 128), bm_, jb + 64 * q, kb * BK);
+                    } else {
+                        #pragma unroll
+                        for (int h = 0; h < C::B_ROWS / 128; ++h) load(sb + h * (128 * BK * 2), bmap, kb * BK, jb + 128 * h);
                     }
                     issued[stage] = static_cast<int>(phase);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -609,7 +650,6 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
     } else if (warp == 1) {
         // ---------------- MMA issuer (leader CTA) ----------------
         if (lane == 0 && leader) {
-            const uint32_t idesc = make_idesc(gemm, C::TILE_M);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -628,11 +668,18 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
                     const uint32_t sb = sa + A_BYTES;
+                    const int kt = kb / (BN / BK);
+                    const bool a_t = kSymA<ph> && kt < td.tm;           // same choice as the producer's
+                    const bool b_t = gemm || (kSymB<ph> && kt < td.tn);
+                    const uint32_t idesc = make_idesc(a_t, b_t, C::TILE_M);
                     #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024);
-                        const uint64_t bd = gemm ? smem_desc(sb + kk * 16 * 128, BK * 128, 1024)
-                                                 : smem_desc(sb + kk * 32, 16, 1024);
+                        // K-major: 16 K columns = 32 B further along each row; MN-major: 16 K rows
+                        // of 128 B further, 64-wide MN chunks BK * 128 B apart
+                        const uint64_t ad = a_t ? smem_desc(sa + kk * 16 * 128, BK * 128, 1024)
+                                                : smem_desc(sa + kk * 32, 16, 1024);
+                        const uint64_t bd = b_t ? smem_desc(sb + kk * 16 * 128, BK * 128, 1024)
+                                                : smem_desc(sb + kk * 32, 16, 1024);
                         if (CG == 2) tc_mma2(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
                         else tc_mma(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
@@ -685,7 +732,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                 if constexpr (gemm)
                     x_load_half(md, iter & 1, gi0, gj_tile, q0, 0, Mrows, Ncols, lane, pre_h, pre_l);
                 else
-                    sym_load_half<ph>(md, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, lane, pre_e, pre_dj);
+                    sym_load_half<ph>(md, td.tm != td.tn, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, lane, pre_e, pre_dj);
             }
             bool ok = true;
             if (lane == 0) ok = wait_bounded(tfull0 + 8 * acc, acc_phase, abort_flag, status);
@@ -700,8 +747,8 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                     epilogue_x_warp(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_h,
                                     pre_l);
                 else
-                    epilogue_sym_warp<ph>(md, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_e,
-                                          pre_dj);
+                    epilogue_sym_warp<ph>(md, sc, sg, td.tm != td.tn, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg,
+                                          lane, pre_e, pre_dj);
             }
             tc_fence_before();
             __syncwarp();
@@ -802,6 +849,8 @@ bool tc_encode_maps(const std::vector<MatDev>& mats, void* host_out) {
         }
         if (!encode_2d(&mp.ea, m.ab, m.r, m.r, m.lda, BK, BM)) return false;
         if (!encode_2d(&mp.eb, m.bm, m.r, m.r, m.lda, BK, BM)) return false;
+        if (!encode_2d(&mp.eat, m.ab, m.r, m.r, m.lda, 64, BK)) return false;
+        if (!encode_2d(&mp.ebt, m.bm, m.r, m.r, m.lda, 64, BK)) return false;
     }
     return true;
 }
