@@ -95,8 +95,12 @@ def test_iteration_counts(ns_steps, mode):
     hs = H.host_state(wl, wl.matrices)
     res = H.gpu_step(hs, mode, ns_steps=ns_steps)
     for k in range(3):
-        H.assert_parity(H.compare_matrix(hs, res, k, mode, ns_steps=ns_steps), mode,
-                        f"ns_steps={ns_steps} {hs.specs[k].rows}x{hs.specs[k].cols}")
+        m = H.compare_matrix(hs, res, k, mode, ns_steps=ns_steps)
+        H.assert_parity(m, mode, f"ns_steps={ns_steps} {hs.specs[k].rows}x{hs.specs[k].cols}")
+        if mode == "bf16" and ns_steps == 0:
+            # no GEMM ran: O is the normalised momentum read back from the bf16
+            # hi + lo master, which holds each element within 2^-16 of itself
+            assert m["rel_O"] <= 2e-5, f"two-part master error {m['rel_O']:.3e}"
 
 
 def test_plain_momentum_and_other_hparams():
