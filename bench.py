@@ -76,9 +76,9 @@ def ns_flops_dense(specs, steps: int = 5) -> float:
 
 
 # Per-launch DRAM bytes of the GEMM phases at the 7B share, from ncu on the
-# 4-matrix case: GRAM 0.594 GB x 6.54, POLY 0.249 GB x 7.0, APPLY 1.658 GB x 6.54,
+# 4-matrix case: GRAM 0.537 GB x 6.54, POLY 0.110 GB x 7.0, APPLY 1.154 GB x 6.54,
 # averaged over 5 GRAM + 5 POLY + 5 APPLY/FINAL launches.
-GEMM_TRAFFIC_7B = round((5 * 0.594e9 * 6.54 + 5 * 0.249e9 * 7.0 + 5 * 1.658e9 * 6.54) / 15)
+GEMM_TRAFFIC_7B = round((5 * 0.537e9 * 6.54 + 5 * 0.110e9 * 7.0 + 5 * 1.154e9 * 6.54) / 15)
 
 
 def split_groups(specs, n_groups: int) -> List[List[int]]:
