@@ -103,15 +103,17 @@ __device__ __forceinline__ T block_sum(T v, T* smem) {
 // ---------------------------------------------------------------------------
 // K1: one 64 x 64 tile of M per block of 256 threads.
 //   buf <- beta buf + (1-beta) G ;  M <- (1-beta) G + beta buf  (or M <- buf)
-// writes buf and X = M, or M^T when rows > cols (bf16 mode: hi part, which is
-// the first GEMM operand, and remainder; fp32 mode: fp32); each tile's sum of
-// M^2 goes to partials[tile].
+// writes buf and X = M, or M^T when rows > cols (bf16 mode: hi and lo parts,
+// the hi part being the first GEMM operand; fp32 mode: fp32).  A block handles
+// kMomGroup tiles of one matrix and writes the group's sum of M^2 to
+// partials[group].  Untransposed tiles run without block barriers; transposed
+// ones alternate between two staging tiles, one barrier each.
 // ---------------------------------------------------------------------------
 template <bool PARTS>
 __global__ void __launch_bounds__(256, 4)
 momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
                 float* __restrict__ partials, int32_t* status) {
-    __shared__ float tileM[kMomTile][kMomTile + 1];
+    __shared__ float tileM2[2][kMomTile][kMomTile + 1];
     __shared__ float red[8];
     const int grp = blockIdx.x;
     const int mi = find_matrix(mats, nmats, grp);
@@ -123,15 +125,17 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     const void* gradp = md.grad;
     const void* const* parts = md.gparts;   // owner-segment contributions (nparts > 0)
     const int nparts = md.nparts;
-    const int mom_vec = md.mom_vec, tiles_n = md.mom_tiles_n, tile0 = md.mom_tile0, grp0 = md.mom_grp0;
+    const int mom_vec = md.mom_vec, tiles_n = md.mom_tiles_n, grp0 = md.mom_grp0;
     const int64_t ntiles = tiles_m * md.mom_tiles_n;
     if (grp < grp0) {  // cannot happen with a host-built table
         record_status(status, -7);
         return;
     }
+    float sumsq = 0.f;
     for (int k = 0; k < kMomGroup; ++k) {
     const int local = (grp - grp0) * kMomGroup + k;
     if (local >= ntiles) break;      // block-uniform
+    float (*tileM)[kMomTile + 1] = tileM2[k & 1];
     const int ti = local / tiles_n, tj = local % tiles_n;
     const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;
     const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
@@ -141,7 +145,6 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     __nv_bfloat16* __restrict__ xb = md.xb[0];  // bf16 mode: hi part ...
     __nv_bfloat16* __restrict__ xl = md.xlo[0]; // ... and lo part
     const int64_t ldx = md.ldx;
-    float sumsq = 0.f;
 
     if (full && mom_vec) {
         // all eight 16-byte loads of this thread are issued before any store
@@ -243,13 +246,12 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
             }
         }
     }
-    const float tot = block_sum(sumsq, red);
-    if (threadIdx.x == 0) partials[tile0 + local] = tot;
-    __syncthreads();                 // red and tileM are reused by the next tile
     }
+    const float tot = block_sum(sumsq, red);
+    if (threadIdx.x == 0) partials[grp] = tot;
 }
 
-// K2: s = 1 / (||M||_F + eps) per matrix; fixed-order fp64 sum of the tile partials.
+// K2: s = 1 / (||M||_F + eps) per matrix; fixed-order fp64 sum of the group partials.
 __global__ void __launch_bounds__(256)
 norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict__ partials,
             float* __restrict__ s_out, float eps) {
@@ -258,8 +260,9 @@ norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict_
     if (mi >= nmats) return;
     const MatDev& md = mats[mi];
     const int64_t tiles = ((md.rows + kMomTile - 1) / kMomTile) * md.mom_tiles_n;
+    const int64_t groups = (tiles + kMomGroup - 1) / kMomGroup;
     double acc = 0.0;
-    for (int64_t t = threadIdx.x; t < tiles; t += blockDim.x) acc += (double)partials[md.mom_tile0 + t];
+    for (int64_t g = threadIdx.x; g < groups; g += blockDim.x) acc += (double)partials[md.mom_grp0 + g];
     const double tot = block_sum(acc, red);
     if (threadIdx.x == 0) s_out[mi] = (float)(1.0 / (sqrt(tot) + (double)eps));
 }
