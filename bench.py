@@ -20,6 +20,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 from typing import Dict, List, Optional
@@ -153,7 +154,9 @@ class ClockSampler:
 
     def __init__(self, gpu_index: Optional[str]):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # raw samples: $MFSDP_CLOCKS_DIR (default: the temporary directory)
+        out_dir = os.environ.get("MFSDP_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"clocks_{os.getpid()}.csv")
         self.gpu_index = gpu_index
 
     def start(self):
