@@ -8,7 +8,7 @@
 
 namespace mfsdp {
 
-// true when the bf16 phases run on the tcgen05 engine of this build
+// true when the bf16 phases run on the tcgen05 engine (compiled for sm_100a)
 bool tc_available();
 
 // bytes of the per-matrix TMA descriptor table (64-byte aligned entries)
