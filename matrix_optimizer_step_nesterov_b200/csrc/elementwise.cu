@@ -277,7 +277,8 @@ norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict_
 __global__ void __launch_bounds__(256, 4)
 param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, const float* __restrict__ s,
                    int xsel, int use_s, int32_t* status) {
-    __shared__ float tileX[kMomTile][kMomTile + 1];
+    // transposed tiles alternate between two staging tiles: one block barrier per tile
+    __shared__ float tileX2[2][kMomTile][kMomTile + 1];
     const int grp = blockIdx.x;
     const int mi = find_matrix(mats, nmats, grp);
     const MatDev& md = mats[mi];
@@ -314,6 +315,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
     for (int k = 0; k < kMomGroup; ++k) {
     const int local = (grp - grp0) * kMomGroup + k;
     if (local >= ntiles) break;      // block-uniform
+    const int sb = k & 1;            // staging tile of this tile
     const int ti = local / tiles_n, tj = local % tiles_n;
     const int64_t i0 = (int64_t)ti * kMomTile, j0 = (int64_t)tj * kMomTile;   // W tile origin
     const bool full = (i0 + kMomTile <= rows) && (j0 + kMomTile <= cols);
@@ -332,9 +334,9 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
                 const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
                 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    tileX[xr][xc + 2 * u] = master_value(static_cast<uint16_t>(hw[u] & 0xFFFFu),
+                    tileX2[sb][xr][xc + 2 * u] = master_value(static_cast<uint16_t>(hw[u] & 0xFFFFu),
                                                          static_cast<uint16_t>(lw[u] & 0xFFFFu));
-                    tileX[xr][xc + 2 * u + 1] = master_value(static_cast<uint16_t>(hw[u] >> 16),
+                    tileX2[sb][xr][xc + 2 * u + 1] = master_value(static_cast<uint16_t>(hw[u] >> 16),
                                                              static_cast<uint16_t>(lw[u] >> 16));
                 }
             }
@@ -363,7 +365,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
                 const int v = e * 256 + threadIdx.x;
                 const int row = v >> 3, col = (v & 7) * 8;
                 #pragma unroll
-                for (int u = 0; u < 8; ++u) xv[e][u] = tileX[col + u][row];
+                for (int u = 0; u < 8; ++u) xv[e][u] = tileX2[sb][col + u][row];
             }
         }
         #pragma unroll
@@ -391,7 +393,6 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
             }
             for (int d = 0; d < ncopies; ++d) *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(copies[d]) + widx) = out;
         }
-        __syncthreads();             // tileX is reused by the next tile
         continue;
     }
     if (tr) {
@@ -403,7 +404,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
                 const int xr = v >> 4, xc = (v & 15) * 4;
                 const int64_t xi = (j0 + xr) * ldx + i0 + xc;
                 const float4 x = bfm ? load4_master(xb, xl, xi) : *reinterpret_cast<const float4*>(xf + xi);
-                tileX[xr][xc] = x.x; tileX[xr][xc + 1] = x.y; tileX[xr][xc + 2] = x.z; tileX[xr][xc + 3] = x.w;
+                tileX2[sb][xr][xc] = x.x; tileX2[sb][xr][xc + 1] = x.y; tileX2[sb][xr][xc + 2] = x.z; tileX2[sb][xr][xc + 3] = x.w;
             }
         } else {
             for (int e = 0; e < 16; ++e) {
@@ -411,7 +412,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
                 const int xr = v >> 6, xc = v & 63;
                 if (j0 + xr < cols && i0 + xc < rows) {
                     const int64_t xi = (j0 + xr) * ldx + i0 + xc;
-                    tileX[xr][xc] = bfm ? load1_master(xb, xl, xi) : xf[xi];
+                    tileX2[sb][xr][xc] = bfm ? load1_master(xb, xl, xi) : xf[xi];
                 }
             }
         }
@@ -424,7 +425,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
         for (int e = 0; e < 4; ++e) {
             const int v = e * 256 + threadIdx.x;
             const int row = v >> 4, col = (v & 15) * 4;
-            if (tr) xv[e] = make_float4(tileX[col][row], tileX[col + 1][row], tileX[col + 2][row], tileX[col + 3][row]);
+            if (tr) xv[e] = make_float4(tileX2[sb][col][row], tileX2[sb][col + 1][row], tileX2[sb][col + 2][row], tileX2[sb][col + 3][row]);
             else if (bfm) xv[e] = load4_master(xb, xl, (i0 + row) * ldx + j0 + col);
             else xv[e] = *reinterpret_cast<const float4*>(xf + (i0 + row) * ldx + j0 + col);
             wv[e] = load4(md.param, (i0 + row) * cols + j0 + col, wbf);
@@ -452,7 +453,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
         const int row = v >> 6, col = v & 63;
         const int64_t i = i0 + row, j = j0 + col;
         if (i >= rows || j >= cols) continue;
-        const float x = tr ? tileX[col][row] : (bfm ? load1_master(xb, xl, i * ldx + j) : xf[i * ldx + j]);
+        const float x = tr ? tileX2[sb][col][row] : (bfm ? load1_master(xb, xl, i * ldx + j) : xf[i * ldx + j]);
         const float o = f * x;
         const int64_t idx = i * cols + j;
         if (uo) uo[idx] = o;
@@ -467,7 +468,6 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
         }
     }
     }
-    __syncthreads();                 // tileX is reused by the next tile
     }
 }
 
