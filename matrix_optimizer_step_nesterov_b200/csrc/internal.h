@@ -61,8 +61,9 @@ struct TileDev {
 // In bf16 mode this keeps the large diagonal terms (and the near-cancellation
 // a X + D_B X) out of bf16 rounding; the GEMM work is unchanged.
 enum Phase : int32_t {
-    PH_GRAM = 0,   // A = s^2 X X^T -> E_A, d_A                          (upper tiles, mirrored)
-    PH_POLY = 1,   // B = b A + c A A -> E_B operand, d_B                (upper tiles, mirrored)
+    PH_GRAM = 0,   // A = s^2 X X^T -> E_A, d_A          (upper tiles; tensor-core engine: block-upper
+                   //                                      storage, the SIMT engine mirrors)
+    PH_POLY = 1,   // B = b A + c A A -> E_B operand, d_B  (likewise)
     PH_APPLY = 2,  // X <- s ((a + d_B,i) X + E_B X)
     PH_FINAL = 3,  // the last iteration's X update (the same arithmetic); the parameter
                    // write then runs as its own HBM-bound kernel
