@@ -331,9 +331,11 @@ def run_ours(args) -> int:
     if world > 1:
         dist.barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_steps = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev0.record(stream)
-    for _ in range(args.steps):
+    for k in range(args.steps):
         one_step()
+        ev_steps[k].record(stream)           # per-step boundaries, for the median and minimum
     ev1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -342,6 +344,11 @@ def run_ours(args) -> int:
     clocks = sampler.stop() if sampler else None
     ms_local = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms_local)
+    per_step = [ev0.elapsed_time(ev_steps[0])] + [ev_steps[k - 1].elapsed_time(ev_steps[k])
+                                                  for k in range(1, args.steps)]
+    step_stats = {"median_ms": round(max_over_ranks(statistics.median(per_step)), 4),
+                  "min_ms": round(max_over_ranks(min(per_step)), 4),
+                  "max_ms": round(max_over_ranks(max(per_step)), 4)}
 
     # e2e through host buffers: every gradient in (pinned H2D) and every updated
     # parameter out (D2H) each step.  The owner's matrices are split into
@@ -522,6 +529,7 @@ def run_ours(args) -> int:
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms, 4),
+        "step_ms": step_stats,
         "higher_is_better": False,
         "scaling": "weak",
         "vs_baseline": None,
