@@ -119,7 +119,11 @@ def bench_workload(args):
         dtype = "bf16" if args.mode == "bf16" else "f32"
         return custom_workload(shapes, dtype=dtype, tail=args.tail, seed=4242, spike_rule="rank:4:rel:10",
                                name="shapes " + args.shapes)
-    return workload(args.workload)
+    wl = workload(args.workload)
+    if args.seed is not None:                # a second draw of the same workload
+        import dataclasses
+        wl = dataclasses.replace(wl, seed=args.seed)
+    return wl
 
 
 def max_over_ranks(x: float) -> float:
@@ -611,6 +615,7 @@ def main(argv=None) -> int:
     ap.add_argument("--mode", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--shapes", default="", help="explicit matrix list RxC,RxC (profiling cases) instead of --workload")
     ap.add_argument("--tail", type=int, default=0, help="tail length with --shapes")
+    ap.add_argument("--seed", type=int, default=None, help="input seed instead of the workload's own")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-groups", type=int, default=6, help="matrix groups pipelined in the e2e measurement")

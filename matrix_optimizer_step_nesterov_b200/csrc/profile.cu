@@ -1,6 +1,10 @@
-// Per-kernel-class CUDA-event timing of the library's own launches.
+// Per-kernel-class CUDA-event timing of the library's own launches, and an
+// NVTX range named after the kernel class around every launch (free unless a
+// profiler is attached).
 #include "../../include/mfsdp.h"
 #include "internal.h"
+
+#include <nvtx3/nvToolsExt.h>
 
 #include <mutex>
 #include <vector>
@@ -21,7 +25,13 @@ int g_used = 0;
 
 }  // namespace
 
+const char* const kRangeNames[MFSDP_KCLASS_COUNT] = {
+    "mfsdp:momentum", "mfsdp:norm", "mfsdp:gram", "mfsdp:poly",
+    "mfsdp:apply", "mfsdp:write", "mfsdp:adamw", "mfsdp:final",
+};
+
 int prof_before(int cls, cudaStream_t s) {
+    nvtxRangePushA((cls >= 0 && cls < MFSDP_KCLASS_COUNT) ? kRangeNames[cls] : "mfsdp");
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_active || g_used >= g_capacity) return -1;
     Slot& sl = g_slots[g_used];
@@ -34,6 +44,7 @@ int prof_before(int cls, cudaStream_t s) {
 }
 
 void prof_after(int slot, cudaStream_t s) {
+    nvtxRangePop();
     if (slot < 0) return;
     std::lock_guard<std::mutex> lock(g_mu);
     if (slot < static_cast<int>(g_slots.size()) && cudaEventRecord(g_slots[slot].stop, s) != cudaSuccess) {
