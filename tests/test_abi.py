@@ -241,3 +241,34 @@ def test_reshard_validation(lib):
     assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
     shards, routes, moved = lib.mfsdp_reshard([], [], 3)
     assert shards == [] and routes == [] and moved == 0
+
+
+def test_planner_and_reshard_match_oracle_on_random_lists(lib):
+    # seeded random parameter lists: mixed dtypes, tall and wide matrices, tails,
+    # repeated shapes (ties), world sizes 1..9
+    import numpy as np
+    from synth.workloads import ParamSpec, TAIL
+    rng = np.random.default_rng(20261202)
+    for trial in range(40):
+        n = int(rng.integers(1, 30))
+        params = []
+        for pid in range(n):
+            if rng.random() < 0.15:
+                params.append(ParamSpec(pid, f"t{pid}", int(rng.integers(1, 5000)), 1, TAIL, "f32"))
+            else:
+                r = int(rng.choice([64, 128, 96, 4096, 11008, 5120, 1]) if rng.random() < 0.5 else rng.integers(1, 700))
+                c = int(rng.choice([64, 128, 4096, 2048]) if rng.random() < 0.5 else rng.integers(1, 700))
+                params.append(ParamSpec(pid, f"m{pid}", r, c, MATRIX, "bf16" if rng.random() < 0.7 else "f32"))
+        descs = [(p.rows, p.cols, p.kind, 1 if p.dtype == "bf16" else 0) for p in params]
+        R = int(rng.integers(1, 10))
+        shards, F, B = lib.mfsdp_plan(descs, R)
+        entries, Fo, Bo = oracle.plan_owners(params, R)
+        assert [(s.owner, s.owner_offset) for s in shards] == [(e.owner, e.owner_offset) for e in entries], trial
+        assert F == Fo and B == Bo, trial
+        R2 = int(rng.integers(1, 10))
+        new, routes, moved = lib.mfsdp_reshard(descs, shards, R2)
+        new_o, routes_o, moved_o = oracle.reshard(params, entries, R2)
+        assert [(s.owner, s.owner_offset) for s in new] == [(e.owner, e.owner_offset) for e in new_o], trial
+        assert [(r.src_rank, r.src_offset, r.dst_rank, r.dst_offset, r.state_bytes) for r in routes] == \
+            [(o.src_rank, o.src_offset, o.dst_rank, o.dst_offset, o.state_bytes) for o in routes_o], trial
+        assert moved == moved_o, trial
