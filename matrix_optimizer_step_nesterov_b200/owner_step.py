@@ -114,6 +114,16 @@ class MuonOwnerStep:
             _lib.mfsdp_muon_step(self.mats, self.hp, self.workspace_ptr, self.workspace_bytes,
                                  _stream_handle(stream), arr=self._arr)
 
+    def capture_graph(self) -> "torch.cuda.CUDAGraph":
+        """One step captured into a CUDA graph; ``replay()`` reruns it on the same
+        tensors with the same hyper-parameters.  Call ``step()`` once before
+        capturing: the workspace's descriptor table is then already on the
+        device, and the capture holds only the step's kernel launches."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step()
+        return g
+
     def close(self) -> None:
         if getattr(self, "_ws", None) is not None:
             _lib.mfsdp_muon_forget_workspace(self.workspace_ptr)

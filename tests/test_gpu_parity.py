@@ -205,3 +205,36 @@ def test_adamw_skew_tail_sampled():
     p, m, v = H.gpu_adamw(ti.p, ti.g, ti.m, ti.v, 10)
     pr, mr, vr = oracle.adamw_step(ti.p, ti.g, ti.m, ti.v, 10, H.adamw_hparams_as_passed())
     assert H.adamw_tolerance_ok(p, pr) and H.adamw_tolerance_ok(m, mr) and H.adamw_tolerance_ok(v, vr)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_cuda_graph_replay_matches_eager_steps(mode):
+    # two eager steps against one eager step plus the replay of a captured step:
+    # the same launches on the same buffers, so the results are bit-identical
+    import torch
+    from matrix_optimizer_step_nesterov_b200 import MuonOwnerStep
+    wl = custom_workload([(300, 520), (520, 300), (64, 64)], dtype="f32" if mode == "fp32" else "bf16", seed=11)
+    hs = H.host_state(wl, wl.matrices, buf_init="random")
+    dev = torch.device("cuda")
+    dt = torch.float32 if mode == "fp32" else torch.bfloat16
+
+    def make():
+        ps = [torch.from_numpy(w).to(dt).to(dev) for w in hs.W]
+        gs = [torch.from_numpy(g).to(dt).to(dev) for g in hs.G]
+        bs = [torch.from_numpy(b).to(dev) for b in hs.buf]
+        return ps, gs, bs, MuonOwnerStep(ps, gs, bs, mode=mode)
+
+    pa, ga, ba, sa = make()
+    sa.step()
+    sa.step()
+    pb, gb, bb, sb = make()
+    sb.step()
+    g = sb.capture_graph()
+    g.replay()
+    torch.cuda.synchronize()
+    for k in range(len(pa)):
+        assert torch.equal(pa[k], pb[k]), f"param {k}"
+        assert torch.equal(ba[k], bb[k]), f"momentum {k}"
+    del g
+    sa.close()
+    sb.close()
