@@ -163,6 +163,42 @@ void build_tiles(Layout& L, Engine eng) {
     L.poly_tiles = L.sym_tiles;
 }
 
+// Self-check of the host-built tile tables: every output tile of every matrix
+// appears exactly once - all tiles of X for the general phase, the tiles that
+// reach the upper triangle of the r x r result for GRAM and POLY - with a
+// positive K depth.  A failure is a bug in the tile builder, never the caller's.
+bool tiles_cover(const Layout& L, int tm_edge, int tn_edge) {
+    const int32_t nm = static_cast<int32_t>(L.mats.size());
+    auto check = [&](const std::vector<TileDev>& tiles, bool sym) {
+        std::vector<size_t> base(static_cast<size_t>(nm) + 1, 0);
+        std::vector<int> ncols(static_cast<size_t>(nm), 0), nrows(static_cast<size_t>(nm), 0);
+        for (int32_t i = 0; i < nm; ++i) {
+            const MatDev& m = L.mats[i];
+            nrows[i] = (m.r + tm_edge - 1) / tm_edge;
+            ncols[i] = ((sym ? m.r : m.c) + tn_edge - 1) / tn_edge;
+            base[i + 1] = base[i] + static_cast<size_t>(nrows[i]) * ncols[i];
+        }
+        std::vector<uint8_t> seen(base[nm], 0);
+        for (const TileDev& t : tiles) {
+            if (t.mat < 0 || t.mat >= nm || t.kblk <= 0) return false;
+            if (t.tm < 0 || t.tm >= nrows[t.mat] || t.tn < 0 || t.tn >= ncols[t.mat]) return false;
+            if (sym && static_cast<int64_t>(t.tm) * tm_edge > static_cast<int64_t>(t.tn) * tn_edge + tn_edge - 1)
+                return false;
+            uint8_t& c = seen[base[t.mat] + static_cast<size_t>(t.tm) * ncols[t.mat] + t.tn];
+            if (c) return false;
+            c = 1;
+        }
+        for (int32_t i = 0; i < nm; ++i)
+            for (int a = 0; a < nrows[i]; ++a)
+                for (int b = 0; b < ncols[i]; ++b) {
+                    const bool wanted = !sym || static_cast<int64_t>(a) * tm_edge <= static_cast<int64_t>(b) * tn_edge + tn_edge - 1;
+                    if (seen[base[i] + static_cast<size_t>(a) * ncols[i] + b] != (wanted ? 1 : 0)) return false;
+                }
+        return true;
+    };
+    return check(L.sym_tiles, true) && check(L.poly_tiles, true) && check(L.gen_tiles, false);
+}
+
 int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32_t n,
                  const mfsdp_muon_hparams* hp, char* base, Layout& L) {
     const bool bf16 = hp->mode == MFSDP_MODE_BF16;
@@ -217,6 +253,9 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
     L.mom_tiles = tile0;
     L.mom_groups = grp0;
     build_tiles(L, L.engine);
+    if (L.engine == Engine::Tc ? !tiles_cover(L, tc_tile_rows(), tc_tile_cols())
+                               : !tiles_cover(L, kSimtTile, kSimtTile))
+        return MFSDP_ERR_INVALID_ARG;
     const size_t nm = L.mats.size();
     size_t off = 0;
     L.off_mats = off;      off = align_up(off + nm * sizeof(MatDev));

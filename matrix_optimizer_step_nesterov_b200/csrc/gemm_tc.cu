@@ -838,6 +838,9 @@ cudaError_t launch_bounded_wait_selftest(unsigned long long limit_ns, cudaStream
 
 size_t tc_maps_bytes(size_t nmats) { return nmats * sizeof(TcMaps); }
 
+int tc_tile_rows() { return TcCfg<kCtaGroup>::TILE_M; }
+int tc_tile_cols() { return BN; }
+
 bool tc_encode_maps(const std::vector<MatDev>& mats, void* host_out) {
     TcMaps* out = static_cast<TcMaps*>(host_out);
     for (size_t i = 0; i < mats.size(); ++i) {

@@ -22,6 +22,10 @@ bool tc_encode_maps(const std::vector<MatDev>& mats, void* host_out);
 void tc_build_tiles(const std::vector<MatDev>& mats, std::vector<TileDev>& gram, std::vector<TileDev>& poly,
                     std::vector<TileDev>& gen);
 
+// output tile edges of the engine's tiles (rows of a tile, columns of a tile)
+int tc_tile_rows();
+int tc_tile_cols();
+
 // one CTA whose single wait runs out after limit_ns (failure-detection test)
 cudaError_t launch_bounded_wait_selftest(unsigned long long limit_ns, cudaStream_t st);
 

@@ -272,3 +272,23 @@ def test_planner_and_reshard_match_oracle_on_random_lists(lib):
         assert [(r.src_rank, r.src_offset, r.dst_rank, r.dst_offset, r.state_bytes) for r in routes] == \
             [(o.src_rank, o.src_offset, o.dst_rank, o.dst_offset, o.state_bytes) for o in routes_o], trial
         assert moved == moved_o, trial
+
+
+def test_tile_tables_cover_every_output_tile_once(lib):
+    # mfsdp_muon_workspace_size builds the step's tile tables on the host and
+    # rejects any table that misses or repeats an output tile; exercise it on
+    # seeded random lists (ragged edges, r = 1, tall and wide) in both engines
+    import numpy as np
+    rng = np.random.default_rng(7)
+    for trial in range(60):
+        mats = []
+        base = 1 << 20
+        for i in range(int(rng.integers(1, 12))):
+            r = int(rng.choice([1, 63, 64, 255, 256, 257, 600, 1100, 4096]))
+            c = int(rng.choice([1, 64, 129, 256, 513, 2049, 11008]))
+            mats.append(lib.Matrix(base, base + (1 << 28), base + (2 << 28), None, r, c, 1, 1))
+            base += 3 << 28
+        for mode in (lib.MFSDP_MODE_BF16, lib.MFSDP_MODE_FP32):
+            ms = mats if mode == lib.MFSDP_MODE_BF16 else [
+                lib.Matrix(m.param, m.grad, m.momentum, None, m.rows, m.cols, 0, 0) for m in mats]
+            assert lib.mfsdp_muon_workspace_size(ms, lib.muon_hparams(mode=mode)) > 0, trial
