@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <unordered_map>
 #include <vector>
@@ -25,23 +26,23 @@ size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
 
 int check_device() {
-    static int cached[64] = {0};  // 0 unknown, 1 ok, -1 unsupported
+    static std::atomic<int> cached[64];  // 0 unknown, 1 ok, -1 unsupported (zero-initialised)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return MFSDP_ERR_CUDA;
     }
     if (dev < 0 || dev >= 64) return MFSDP_ERR_UNSUPPORTED_DEVICE;
-    if (cached[dev] == 0) {
+    if (cached[dev].load(std::memory_order_relaxed) == 0) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
             cudaGetLastError();
             return MFSDP_ERR_CUDA;
         }
-        cached[dev] = (major == 10 && minor == 0) ? 1 : -1;
+        cached[dev].store((major == 10 && minor == 0) ? 1 : -1, std::memory_order_relaxed);
     }
-    return cached[dev] == 1 ? MFSDP_OK : MFSDP_ERR_UNSUPPORTED_DEVICE;
+    return cached[dev].load(std::memory_order_relaxed) == 1 ? MFSDP_OK : MFSDP_ERR_UNSUPPORTED_DEVICE;
 }
 
 bool aligned(const void* p, size_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }

@@ -527,13 +527,16 @@ adamw_scalar_kernel(float* __restrict__ p, const float* __restrict__ g, float* _
 }
 
 int sm_count() {
-    static int count = 0;
-    if (count == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
-        if (count <= 0) count = 148;
-    }
+    // initialised once, thread-safely, on the first call
+    static const int count = [] {
+        int dev = 0, c = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) {
+            cudaGetLastError();
+            c = 148;
+        }
+        return c;
+    }();
     return count;
 }
 
@@ -574,14 +577,14 @@ cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, int64_t n
     const int64_t work = vec ? n / 4 : n;
     int64_t blocks = (work + 4 * 256 - 1) / (4 * 256);
     // a grid of resident blocks only: the grid-stride loop then has no tail wave
-    static int per_sm = 0;
-    if (per_sm == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adamw_vec_kernel, 256, 0) != cudaSuccess ||
-            per_sm <= 0) {
+    static const int per_sm = [] {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, adamw_vec_kernel, 256, 0) != cudaSuccess || n <= 0) {
             cudaGetLastError();
-            per_sm = 2;
+            n = 2;
         }
-    }
+        return n;
+    }();
     const int64_t cap = (int64_t)sm_count() * per_sm;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;

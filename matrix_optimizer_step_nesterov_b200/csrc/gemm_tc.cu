@@ -903,14 +903,10 @@ cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats
                          int32_t ntiles, int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st,
                          int sms) {
     constexpr int CG = kCtaGroup;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(tc_phase_kernel<ph, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   TcCfg<CG>::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    static int max_clusters = 0;      // clusters of CG CTAs that fit on the device at once
+    // one-time, thread-safe set-up of this phase's kernel
+    static const cudaError_t attr_err = cudaFuncSetAttribute(
+        tc_phase_kernel<ph, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<CG>::SMEM_BYTES);
+    if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((sms / CG) * CG, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -923,14 +919,15 @@ cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (max_clusters == 0) {
+    // clusters of CG CTAs that fit on the device at once (computed once)
+    static const int max_clusters = [&] {
         int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, tc_phase_kernel<ph, CG>, &cfg) != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = sms / CG;
         }
-        max_clusters = n;
-    }
+        return n;
+    }();
     const int clusters = std::max(1, std::min(ntiles, max_clusters));
     cfg.gridDim = dim3(clusters * CG, 1, 1);
     return cudaLaunchKernelEx(&cfg, tc_phase_kernel<ph, CG>, d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s,
@@ -943,13 +940,15 @@ cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, i
                            const TileDev* d_tiles, int32_t ntiles, int32_t iter, const StepScalars& sc,
                            const float* s, cudaStream_t st) {
     if (ntiles <= 0) return cudaSuccess;
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
+    static const int sms = [] {
+        int dev = 0, c = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) {
+            cudaGetLastError();
+            c = 148;
+        }
+        return c;
+    }();
     const TcMaps* maps = static_cast<const TcMaps*>(d_maps);
     cudaError_t e;
     switch (ph) {
