@@ -284,7 +284,8 @@ int mfsdp_muon_forget_workspace(void* workspace);
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  Every call shares the one array, so calls that
  * overlap on the GPU (other streams, other threads) race; serialise them.
- * Nothing in the array needs to start at zero: each call writes what it reads.
+ * Nothing in the array needs to start at zero: every value a call's results
+ * depend on is written by that call before it is read.
  */
 int mfsdp_muon_step_noalloc(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp, void* stream);
 
