@@ -271,10 +271,11 @@ int mfsdp_muon_forget_workspace(void* workspace);
 
 /*
  * mfsdp_muon_step_noalloc - mfsdp_muon_step without a caller workspace, for
- * callers that cannot allocate device memory at step time: code running under
- * CUDA stream capture, hosts that hand out every byte from their own
- * pre-planned pools, loops that must not enter an allocator.  The paper has no
- * counterpart; this is a deployment convenience of this library.
+ * callers that cannot allocate device memory at step time: hosts and plugins
+ * that hand out every byte from their own pre-planned pools and forbid driver
+ * allocations, and loops that must not enter an allocator (which may
+ * synchronise the device).  The paper has no counterpart; this is a
+ * deployment convenience of this library.
  *   mats, n, hp, stream  as for mfsdp_muon_step (same validation, same result)
  * Scratch: a fixed 64 MiB array compiled into the library, one per GPU that
  * loads it, held until process exit.  Lists whose mfsdp_muon_workspace_size()
@@ -282,10 +283,12 @@ int mfsdp_muon_forget_workspace(void* workspace);
  * GPU work.  The call allocates no device memory.
  * The first call on a device resolves the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call shares the one array, so calls that
- * overlap on the GPU (other streams, other threads) race; serialise them.
- * Nothing in the array needs to start at zero: every value a call's results
- * depend on is written by that call before it is read.
+ * before any stream capture.  Every call shares the one array and keeps its
+ * contents until the next call, so calls that overlap on the GPU (other
+ * streams, other threads) race; serialise them.  Each call enqueues the upload
+ * of its own descriptor and tile tables into the array on `stream` before its
+ * kernels, and nothing else in the array needs to start at zero: every value
+ * a call's results depend on is written by that call before it is read.
  */
 int mfsdp_muon_step_noalloc(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp, void* stream);
 

@@ -342,9 +342,6 @@ int workspace_size_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* se
 
 }  // namespace
 
-int muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
-                   const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes, void* stream);
-
 }  // namespace mfsdp
 
 using namespace mfsdp;
@@ -390,7 +387,8 @@ extern "C" int mfsdp_muon_step_p2p(const mfsdp_matrix* mats, const mfsdp_owner_s
 }
 
 int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
-                          const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes, void* stream) {
+                          const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes, void* stream,
+                          bool always_upload) {
     int st = validate_all(mats, segs, n, hp);
     if (st) return st;
     int32_t live = 0;
@@ -424,14 +422,16 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
     {
         std::lock_guard<std::mutex> lock(g_cache_mu);
         auto it = g_cache.find(reinterpret_cast<uintptr_t>(workspace));
-        const bool fresh = it != g_cache.end() && it->second.dev == dev && it->second.head == head;
+        const bool fresh = !always_upload && it != g_cache.end() && it->second.dev == dev && it->second.head == head;
         if (!fresh) {
             if (cudaMemcpyAsync(base, head.data(), head.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) {
                 cudaGetLastError();
                 g_cache.erase(reinterpret_cast<uintptr_t>(workspace));
                 return MFSDP_ERR_CUDA;
             }
-            g_cache[reinterpret_cast<uintptr_t>(workspace)] = CacheEntry{dev, std::move(head)};
+            // a shared scratch (always_upload) is never assumed to still hold this head
+            if (always_upload) g_cache.erase(reinterpret_cast<uintptr_t>(workspace));
+            else g_cache[reinterpret_cast<uintptr_t>(workspace)] = CacheEntry{dev, std::move(head)};
         }
     }
     const MatDev* d_mats = reinterpret_cast<const MatDev*>(base + L.off_mats);

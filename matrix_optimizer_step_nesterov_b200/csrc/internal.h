@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include "../../include/mfsdp.h"
+
 namespace mfsdp {
 
 // Per-matrix record the kernels read from the workspace head.  X is the
@@ -81,6 +83,14 @@ struct StepScalars {
 
 constexpr int kMomTile = 64;   // momentum / parameter-write tile: 64 x 64 elements of M or W
 constexpr int kMomGroup = 4;   // tiles one block of those kernels processes
+
+// The grouped step behind mfsdp_muon_step (segs == nullptr) and mfsdp_muon_step_p2p.
+// always_upload: enqueue the descriptor-table upload on every call instead of
+// skipping it when the workspace is known to hold the same table already (for a
+// scratch that several matrix lists share).
+int muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                   const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes, void* stream,
+                   bool always_upload = false);
 
 // launch timing hooks (profile.cu): slot = prof_before(class, stream); launch; prof_after(slot, stream)
 int prof_before(int cls, cudaStream_t s);

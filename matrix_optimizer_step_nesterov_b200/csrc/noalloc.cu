@@ -1,14 +1,12 @@
 // mfsdp_muon_step_noalloc: the grouped Muon step for callers that cannot
 // allocate device memory.
 //
-// Some callers have no way to obtain a workspace at step time: code that runs
-// while a stream is being captured into a CUDA graph (an allocation there
-// would be baked into, or break, the graph), plugins and inference or
-// training hosts that own every byte of device memory through their own
-// pre-planned pools and forbid driver allocations, and latency-critical loops
-// that must not enter an allocator that may synchronise the device.  This
-// entry point takes the step's scratch from a fixed array compiled into the
-// library instead of from the caller.
+// Some callers have no way to obtain a workspace at step time: plugins and
+// inference or training hosts that own every byte of device memory through
+// their own pre-planned pools and forbid driver allocations, and
+// latency-critical loops that must not enter an allocator, which may
+// synchronise the device.  This entry point takes the step's scratch from a
+// fixed array compiled into the library instead of from the caller.
 //
 // The scratch is kNoAllocScratchBytes (64 MiB) of device memory per GPU that
 // loads the library, held until the process exits.  It fits small owner
@@ -16,7 +14,12 @@
 // per element of its r x r Gram matrix (r = the shorter side), e.g. one
 // 2048 x 1024 or several 512 x 512 matrices.  Larger lists are rejected with
 // MFSDP_ERR_WORKSPACE_TOO_SMALL before any GPU work.
+//
+// Every call shares the one array, so every call re-uploads its own
+// descriptor and tile tables into it (enqueued on the caller's stream before
+// the step's kernels) rather than trusting what an earlier call left there.
 #include "../../include/mfsdp.h"
+#include "internal.h"
 
 #include <cuda_runtime.h>
 
@@ -72,6 +75,8 @@ extern "C" int mfsdp_muon_step_noalloc(const mfsdp_matrix* mats, int32_t n, cons
     st = scratch_address(&scratch);
     if (st != MFSDP_OK) return st;
     // The step writes every scratch byte it later reads (tables, partial sums,
-    // X, A and B buffers), so the previous call's contents need no clearing.
-    return mfsdp_muon_step(mats, n, hp, scratch, kNoAllocScratchBytes, stream);
+    // X, A and B buffers), so the previous call's contents need no clearing;
+    // the tables are uploaded on every call, whatever the previous call left.
+    return mfsdp::muon_step_impl(mats, nullptr, n, hp, scratch, kNoAllocScratchBytes, stream,
+                                 /*always_upload=*/true);
 }

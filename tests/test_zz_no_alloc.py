@@ -1,10 +1,13 @@
 """mfsdp_muon_step_noalloc against mfsdp_muon_step, through the C ABI.
 
-The no-allocation entry point serves callers that cannot allocate device
-memory at step time (stream capture, host-owned memory pools): it runs the
-same step with the library's fixed 64 MiB device scratch instead of a caller
-workspace.  Two calls in a row must match two calls of the workspace entry
-point on the same inputs, within the parity tolerance.  This file is named to
+The no-allocation entry point is for callers that cannot allocate device
+memory at step time (hosts and plugins that own all device memory through
+their own pools, loops that must not enter an allocator): it runs the same
+step with the library's fixed 64 MiB device scratch instead of a caller
+workspace.  It launches the same kernels over the same layout, so its results
+must equal the workspace entry point's bit for bit, call after call, also
+when calls alternate between different matrix lists that share the scratch.
+One result is also checked against the fp64 oracle.  This file is named to
 be collected last, and it also passes alone in a fresh process.
 """
 
@@ -41,41 +44,61 @@ def _mats(lib, W, G, B, O):
                        code[w.dtype], code[g.dtype]) for w, g, b, o in zip(W, G, B, O)]
 
 
+class _Pair:
+    """One matrix list stepped twice over: through a private workspace and
+    through the shared no-allocation scratch, from identical copies of the state."""
+
+    def __init__(self, lib, shapes, mode, seed):
+        self.lib = lib
+        self.dtype = torch.bfloat16 if mode == "bf16" else torch.float32
+        wl = custom_workload(shapes, dtype="bf16" if mode == "bf16" else "f32", seed=seed)
+        self.hs = H.host_state(wl, wl.matrices, buf_init="random")
+        self.ref = _device_state(self.hs, self.dtype)
+        self.new = _device_state(self.hs, self.dtype)
+        self.mats_ref = _mats(lib, *self.ref)
+        self.mats_new = _mats(lib, *self.new)
+        self.hp = lib.muon_hparams(mode=lib.MFSDP_MODE_BF16 if mode == "bf16" else lib.MFSDP_MODE_FP32)
+        self.ws_bytes = lib.mfsdp_muon_workspace_size(self.mats_ref, self.hp)
+        assert 0 < self.ws_bytes <= lib.NOALLOC_SCRATCH_BYTES
+        self.ws = torch.empty(self.ws_bytes + 256, dtype=torch.uint8, device="cuda")
+        self.ws_ptr = (self.ws.data_ptr() + 255) // 256 * 256
+
+    def step(self, stream):
+        self.lib.mfsdp_muon_step(self.mats_ref, self.hp, self.ws_ptr, self.ws_bytes, stream)
+        self.lib.mfsdp_muon_step_noalloc(self.mats_new, self.hp, stream)
+
+    def assert_identical(self, what):
+        for k in range(len(self.mats_ref)):
+            for name, a, b in zip("WGBO", self.ref, self.new):
+                assert torch.equal(a[k], b[k]), f"{what}: matrix {k} {name} differs from the workspace entry point"
+
+    def close(self):
+        self.lib.mfsdp_muon_forget_workspace(self.ws_ptr)
+
+
 @pytest.mark.parametrize("mode", ["fp32", "bf16"])
-def test_noalloc_matches_workspace_entry_point_on_two_calls(mode):
+def test_noalloc_equals_workspace_entry_point_bitwise(mode):
     from matrix_optimizer_step_nesterov_b200 import _lib as lib
-    dtype = torch.bfloat16 if mode == "bf16" else torch.float32
-    shapes = [(256, 512), (384, 128), (100, 300)]
-    wl = custom_workload(shapes, dtype="bf16" if mode == "bf16" else "f32", seed=77)
-    hs = H.host_state(wl, wl.matrices, buf_init="random")
-    hp = lib.muon_hparams(mode=lib.MFSDP_MODE_BF16 if mode == "bf16" else lib.MFSDP_MODE_FP32)
     stream = torch.cuda.current_stream().cuda_stream
-
-    # reference: the workspace entry point, two calls in a row
-    Wr, Gr, Br, Or = _device_state(hs, dtype)
-    mats_r = _mats(lib, Wr, Gr, Br, Or)
-    ws_bytes = lib.mfsdp_muon_workspace_size(mats_r, hp)
-    assert ws_bytes <= lib.NOALLOC_SCRATCH_BYTES
-    ws = torch.empty(ws_bytes + 256, dtype=torch.uint8, device="cuda")
-    ws_ptr = (ws.data_ptr() + 255) // 256 * 256
-    # the no-allocation entry point on an identical copy of the state
-    Wn, Gn, Bn, On = _device_state(hs, dtype)
-    mats_n = _mats(lib, Wn, Gn, Bn, On)
-
-    for call in range(2):
-        lib.mfsdp_muon_step(mats_r, hp, ws_ptr, ws_bytes, stream)
-        lib.mfsdp_muon_step_noalloc(mats_n, hp, stream)
-        torch.cuda.synchronize()
-        for k in range(len(shapes)):
-            o_ref = Or[k].cpu().numpy().astype(np.float64)
-            o_new = On[k].cpu().numpy().astype(np.float64)
-            assert H.rel_frob(o_new, o_ref) <= H.TOL_O[mode], f"call {call} matrix {k}: update differs"
-            assert H.rel_frob(Bn[k].cpu().numpy(), Br[k].cpu().numpy().astype(np.float64)) <= H.TOL_BUF
-            w_ref = Wr[k].cpu().to(torch.float64).numpy()
-            w_new = Wn[k].cpu().to(torch.float64).numpy()
-            assert H.rel_frob(w_new, w_ref) <= H.TOL_O[mode] * 0.02 + 1e-6
-    lib.mfsdp_muon_forget_workspace(ws_ptr)
-    assert lib.mfsdp_get_device_status(stream) == 0
+    a = _Pair(lib, [(256, 512), (384, 128), (100, 300)], mode, seed=77)
+    b = _Pair(lib, [(640, 200), (128, 128), (33, 1000), (513, 257)], mode, seed=78)
+    try:
+        # two calls in a row on list A, then list B, then A again: the shared
+        # scratch holds the other list's tables and buffers between them
+        for call, pair in enumerate((a, a, b, b, a)):
+            pair.step(stream)
+            torch.cuda.synchronize()
+            pair.assert_identical(f"call {call}")
+            if call == 2:
+                # list B's first step, right after list A used the scratch, against the oracle
+                for k in range(len(b.hs.specs)):
+                    _, O_ref, _ = H.oracle_step(b.hs, k)
+                    o_new = b.new[3][k].cpu().numpy().astype(np.float64)
+                    assert H.rel_frob(o_new, O_ref) <= H.TOL_O[mode], f"matrix {k}: update differs from the oracle"
+        assert lib.mfsdp_get_device_status(stream) == 0
+    finally:
+        a.close()
+        b.close()
 
 
 def test_noalloc_rejects_lists_beyond_its_scratch():
