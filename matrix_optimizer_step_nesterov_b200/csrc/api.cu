@@ -120,11 +120,12 @@ int check_no_alias(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, i
     return MFSDP_OK;
 }
 
-// Which GEMM engine runs the Newton-Schulz phases for this call.
+// The GEMM engine of each mode: bf16 operands run on the tcgen05 tensor cores,
+// fp32 mode (no tf32) on the FFMA pipes.  There is no fallback between them.
 enum class Engine { Simt, Tc };
 
 Engine pick_engine(const mfsdp_muon_hparams* hp) {
-    return hp->mode == MFSDP_MODE_BF16 && tc_available() ? Engine::Tc : Engine::Simt;
+    return hp->mode == MFSDP_MODE_BF16 ? Engine::Tc : Engine::Simt;
 }
 
 // Workspace plan: head (descriptor table, tile tables, partials, scales), then
@@ -134,22 +135,35 @@ struct Layout {
     std::vector<TileDev> sym_tiles;    // PH_GRAM
     std::vector<TileDev> poly_tiles;   // PH_POLY
     std::vector<TileDev> gen_tiles;    // PH_APPLY / PH_FINAL
+    // tensor-core engine: each table partitioned over its launch's clusters
+    // (segment offsets, clusters + 1 entries, in a fixed-size head slot)
+    std::vector<int32_t> sym_seg, poly_seg, gen_seg;
     std::vector<uint64_t> ptrs;        // owner-segment part and copy pointers, per matrix
     size_t off_ptrs = 0;
     int32_t mom_tiles = 0;
     int32_t mom_groups = 0;
     size_t off_mats = 0, off_maps = 0, off_sym = 0, off_poly = 0, off_gen = 0, off_partials = 0, off_s = 0;
+    size_t off_sym_seg = 0, off_poly_seg = 0, off_gen_seg = 0;
     size_t head_end = 0, maps_bytes = 0;
     size_t total = 0;
     Engine engine = Engine::Simt;
 };
 
-void build_tiles(Layout& L, Engine eng) {
+// Clusters a persistent phase may use at most; the head reserves room for
+// that many segment offsets per phase, so the layout does not depend on the
+// device.
+constexpr int kMaxClusters = 1024;
+
+void build_tiles(Layout& L, Engine eng, int max_clusters) {
     L.sym_tiles.clear();
     L.poly_tiles.clear();
     L.gen_tiles.clear();
+    L.sym_seg.clear();
+    L.poly_seg.clear();
+    L.gen_seg.clear();
     if (eng == Engine::Tc) {
-        tc_build_tiles(L.mats, L.sym_tiles, L.poly_tiles, L.gen_tiles);
+        tc_build_tiles(L.mats, std::max(1, std::min(max_clusters, kMaxClusters)), L.sym_tiles, L.poly_tiles,
+                       L.gen_tiles, L.sym_seg, L.poly_seg, L.gen_seg);
         return;
     }
     const int T = kSimtTile;
@@ -197,11 +211,25 @@ bool tiles_cover(const Layout& L, int tm_edge, int tn_edge) {
                 }
         return true;
     };
+    // segments: clusters + 1 nondecreasing offsets from 0 to the table's size
+    auto segs_ok = [](const std::vector<int32_t>& seg, size_t ntiles) {
+        if (seg.size() < 2 || seg.size() > static_cast<size_t>(kMaxClusters) + 1) return false;
+        if (seg.front() != 0 || static_cast<size_t>(seg.back()) != ntiles) return false;
+        for (size_t k = 1; k < seg.size(); ++k)
+            if (seg[k] < seg[k - 1]) return false;
+        return true;
+    };
+    if (L.engine == Engine::Tc &&
+        !(segs_ok(L.sym_seg, L.sym_tiles.size()) && segs_ok(L.poly_seg, L.poly_tiles.size()) &&
+          segs_ok(L.gen_seg, L.gen_tiles.size())))
+        return false;
     return check(L.sym_tiles, true) && check(L.poly_tiles, true) && check(L.gen_tiles, false);
 }
 
+// max_clusters: the tensor-core engine's persistent grid on this device (any
+// value >= 1 when only the size is wanted: it changes no offset)
 int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32_t n,
-                 const mfsdp_muon_hparams* hp, char* base, Layout& L) {
+                 const mfsdp_muon_hparams* hp, char* base, Layout& L, int max_clusters) {
     const bool bf16 = hp->mode == MFSDP_MODE_BF16;
     L.engine = pick_engine(hp);
     L.mats.clear();
@@ -253,7 +281,7 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
     }
     L.mom_tiles = tile0;
     L.mom_groups = grp0;
-    build_tiles(L, L.engine);
+    build_tiles(L, L.engine, max_clusters);
     if (L.engine == Engine::Tc ? !tiles_cover(L, tc_tile_rows(), tc_tile_cols())
                                : !tiles_cover(L, kSimtTile, kSimtTile))
         return MFSDP_ERR_INVALID_ARG;
@@ -272,6 +300,10 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
     L.off_sym = off;       off = align_up(off + L.sym_tiles.size() * sizeof(TileDev));
     L.off_poly = off;      off = align_up(off + L.poly_tiles.size() * sizeof(TileDev));
     L.off_gen = off;       off = align_up(off + L.gen_tiles.size() * sizeof(TileDev));
+    const size_t seg_bytes = L.engine == Engine::Tc ? (kMaxClusters + 1) * sizeof(int32_t) : 0;
+    L.off_sym_seg = off;   off = align_up(off + seg_bytes);
+    L.off_poly_seg = off;  off = align_up(off + seg_bytes);
+    L.off_gen_seg = off;   off = align_up(off + seg_bytes);
     L.off_partials = off;  off = align_up(off + static_cast<size_t>(L.mom_tiles) * sizeof(float));
     L.off_s = off;         off = align_up(off + nm * sizeof(float));
     L.head_end = off;
@@ -334,7 +366,7 @@ int workspace_size_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* se
     int st = validate_all(mats, segs, n, hp);
     if (st) return st;
     Layout L;
-    st = build_layout(mats, segs, n, hp, nullptr, L);
+    st = build_layout(mats, segs, n, hp, nullptr, L, 1);
     if (st) return st;
     *bytes = L.mats.empty() ? 0 : L.total;
     return MFSDP_OK;
@@ -398,9 +430,14 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
     if (st) return st;
     if (!workspace) return MFSDP_ERR_INVALID_ARG;
     if (!aligned(workspace, kAlign)) return MFSDP_ERR_MISALIGNED;
+    int max_clusters = 1;
+    if (pick_engine(hp) == Engine::Tc) {
+        max_clusters = tc_max_clusters();
+        if (max_clusters <= 0) return MFSDP_ERR_CUDA;
+    }
     Layout L;
     char* base = static_cast<char*>(workspace);
-    st = build_layout(mats, segs, n, hp, base, L);
+    st = build_layout(mats, segs, n, hp, base, L, max_clusters);
     if (st) return st;
     if (workspace_bytes < L.total) return MFSDP_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -417,6 +454,12 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
         std::memcpy(head.data() + L.off_poly, L.poly_tiles.data(), L.poly_tiles.size() * sizeof(TileDev));
     if (!L.gen_tiles.empty())
         std::memcpy(head.data() + L.off_gen, L.gen_tiles.data(), L.gen_tiles.size() * sizeof(TileDev));
+    auto put_seg = [&](size_t off, const std::vector<int32_t>& seg) {
+        if (!seg.empty()) std::memcpy(head.data() + off, seg.data(), seg.size() * sizeof(int32_t));
+    };
+    put_seg(L.off_sym_seg, L.sym_seg);
+    put_seg(L.off_poly_seg, L.poly_seg);
+    put_seg(L.off_gen_seg, L.gen_seg);
     int dev = 0;
     cudaGetDevice(&dev);
     {
@@ -462,20 +505,26 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     const int32_t nsym = static_cast<int32_t>(L.sym_tiles.size());
     const int32_t ngen = static_cast<int32_t>(L.gen_tiles.size());
-    auto gemm = [&](Phase ph, const TileDev* tiles, int32_t ntiles, int32_t it, int cls) {
+    const int32_t* d_sym_seg = reinterpret_cast<const int32_t*>(base + L.off_sym_seg);
+    const int32_t* d_poly_seg = reinterpret_cast<const int32_t*>(base + L.off_poly_seg);
+    const int32_t* d_gen_seg = reinterpret_cast<const int32_t*>(base + L.off_gen_seg);
+    auto clusters = [](const std::vector<int32_t>& seg) { return static_cast<int32_t>(seg.size()) - 1; };
+    auto gemm = [&](Phase ph, const TileDev* tiles, int32_t ntiles, const int32_t* d_seg, int32_t nclus, int32_t it,
+                    int cls) {
         const int sl = prof_before(cls, s);
         const cudaError_t r = L.engine == Engine::Tc
-                                  ? launch_gemm_tc(ph, d_mats, d_maps, nm, tiles, ntiles, it, sc, d_s, s)
+                                  ? launch_gemm_tc(ph, d_mats, d_maps, nm, tiles, d_seg, nclus, it, sc, d_s, s)
                                   : launch_gemm_simt(ph, d_mats, nm, tiles, ntiles, it, sc, d_s, s);
         prof_after(sl, s);
         return r;
     };
     for (int32_t it = 0; it < hp->ns_steps; ++it) {
         const bool last = it == hp->ns_steps - 1;
-        e = gemm(PH_GRAM, d_sym, nsym, it, MFSDP_KCLASS_GRAM);
-        if (e == cudaSuccess) e = gemm(PH_POLY, d_poly, nsym, it, MFSDP_KCLASS_POLY);
+        e = gemm(PH_GRAM, d_sym, nsym, d_sym_seg, clusters(L.sym_seg), it, MFSDP_KCLASS_GRAM);
+        if (e == cudaSuccess) e = gemm(PH_POLY, d_poly, nsym, d_poly_seg, clusters(L.poly_seg), it, MFSDP_KCLASS_POLY);
         if (e == cudaSuccess)
-            e = gemm(last ? PH_FINAL : PH_APPLY, d_gen, ngen, it, last ? MFSDP_KCLASS_FINAL : MFSDP_KCLASS_APPLY);
+            e = gemm(last ? PH_FINAL : PH_APPLY, d_gen, ngen, d_gen_seg, clusters(L.gen_seg), it,
+                     last ? MFSDP_KCLASS_FINAL : MFSDP_KCLASS_APPLY);
         if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     }
     // the parameter write reads X from the master copy the last iteration wrote

@@ -1,8 +1,8 @@
 // Grouped Newton-Schulz GEMM phases on the FFMA pipe (CUDA cores).
 //
-// This is the fp32 path (MFSDP_MODE_FP32: fp32 operands, no tf32) and the
-// portable fallback of the bf16 path.  One 128 x 128 output tile per block of
-// 256 threads, 8 x 8 accumulators per thread, K staged through double-buffered
+// This is the engine of fp32 mode only (MFSDP_MODE_FP32: fp32 operands, no
+// tf32); bf16 mode always runs on the tcgen05 engine.  One 128 x 128 output
+// tile per block of 256 threads, 8 x 8 accumulators per thread, K staged through double-buffered
 // shared memory 8 deep.  Phases (one launch each, grouped over all matrices):
 //   PH_GRAM   A = s^2 X X^T       upper-triangle tiles, mirrored store
 //   PH_POLY   B = b A + c A A     upper-triangle tiles, mirrored store (A symmetric, so A A = A A^T)
@@ -14,9 +14,6 @@
 // the momentum kernel stores M unnormalised and the scale is folded here.
 #include "internal.h"
 
-#include <cuda_bf16.h>
-#include <type_traits>
-
 namespace mfsdp {
 namespace {
 
@@ -26,14 +23,6 @@ __device__ __forceinline__ float4 ld4(const T* p);
 template <>
 __device__ __forceinline__ float4 ld4<float>(const float* p) {
     return *reinterpret_cast<const float4*>(p);
-}
-
-template <>
-__device__ __forceinline__ float4 ld4<__nv_bfloat16>(const __nv_bfloat16* p) {
-    uint2 raw = *reinterpret_cast<const uint2*>(p);
-    float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw.x));
-    float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw.y));
-    return make_float4(a.x, a.y, b.x, b.y);
 }
 
 __device__ __forceinline__ void mask4(float4& v, int first, int limit) {
@@ -47,19 +36,16 @@ template <typename T>
 __device__ __forceinline__ void store_val(T* p, float v);
 template <>
 __device__ __forceinline__ void store_val<float>(float* p, float v) { *p = v; }
-template <>
-__device__ __forceinline__ void store_val<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
 constexpr int BT = kSimtTile;  // 128
 constexpr int BK = 8;
 constexpr int LDS = BT + 4;
 
-template <bool BF16>
 __global__ void __launch_bounds__(256, 2)
 simt_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, int32_t nmats,
                   const TileDev* __restrict__ tiles, int32_t iter, StepScalars sc,
                   const float* __restrict__ s, int32_t* status) {
-    using T = typename std::conditional<BF16, __nv_bfloat16, float>::type;
+    using T = float;
     __shared__ __align__(16) float As[2][BK][LDS];
     __shared__ __align__(16) float Bs[2][BK][LDS];
 
@@ -78,15 +64,15 @@ simt_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, int32_t nmats,
     int K, Mrows, Ncols;
     const bool gemm = (ph == PH_APPLY || ph == PH_FINAL);
     if (ph == PH_GRAM) {
-        Aop = Bop = BF16 ? reinterpret_cast<const T*>(md.xb[cur]) : reinterpret_cast<const T*>(md.xf[cur]);
+        Aop = Bop = md.xf[cur];
         ldA = ldB = md.ldx; K = md.c; Mrows = Ncols = md.r;
     } else if (ph == PH_POLY) {
-        Aop = Bop = BF16 ? reinterpret_cast<const T*>(md.ab) : reinterpret_cast<const T*>(md.af);
+        Aop = Bop = md.af;
         ldA = ldB = md.lda; K = md.r; Mrows = Ncols = md.r;
     } else {
         Aop = reinterpret_cast<const T*>(md.bm);
         ldA = md.lda;
-        Bop = BF16 ? reinterpret_cast<const T*>(md.xb[cur]) : reinterpret_cast<const T*>(md.xf[cur]);
+        Bop = md.xf[cur];
         ldB = md.ldx; K = md.r; Mrows = md.r; Ncols = md.c;
     }
     const int i0 = t.tm * BT, j0 = t.tn * BT;
@@ -185,14 +171,9 @@ simt_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, int32_t nmats,
                 if (gi == gj) {
                     md.da[gi] = v;
                     md.af[(int64_t)gi * md.lda + gi] = 0.f;
-                    if (BF16) md.ab[(int64_t)gi * md.lda + gi] = __float2bfloat16_rn(0.f);
                 } else {
                     md.af[(int64_t)gi * md.lda + gj] = v;
                     md.af[(int64_t)gj * md.lda + gi] = v;
-                    if (BF16) {
-                        md.ab[(int64_t)gi * md.lda + gj] = __float2bfloat16_rn(v);
-                        md.ab[(int64_t)gj * md.lda + gi] = __float2bfloat16_rn(v);
-                    }
                 }
             } else if (ph == PH_POLY) {
                 if (gi > gj) continue;
@@ -212,14 +193,9 @@ simt_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, int32_t nmats,
                 }
             } else {
                 const int64_t xi = (int64_t)gi * md.ldx + gj;
-                const float xin = md.xf[BF16 ? 0 : cur][xi];
+                const float xin = md.xf[cur][xi];
                 const float v = sg * fmaf(sc.a + md.db[gi], xin, a);
-                if (BF16) {
-                    md.xf[0][xi] = v;
-                    if (ph == PH_APPLY) md.xb[nxt][xi] = __float2bfloat16_rn(v);
-                } else {
-                    md.xf[nxt][xi] = v;
-                }
+                md.xf[nxt][xi] = v;
             }
         }
     }
@@ -230,12 +206,8 @@ simt_phase_kernel(int32_t ph, const MatDev* __restrict__ mats, int32_t nmats,
 cudaError_t launch_gemm_simt(Phase ph, const MatDev* d_mats, int32_t nmats, const TileDev* d_tiles, int32_t ntiles,
                              int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st) {
     if (ntiles <= 0) return cudaSuccess;
-    if (sc.bf16_mode)
-        simt_phase_kernel<true><<<ntiles, 256, 0, st>>>(ph, d_mats, nmats, d_tiles, iter, sc, s,
-                                                       device_status_ptr());
-    else
-        simt_phase_kernel<false><<<ntiles, 256, 0, st>>>(ph, d_mats, nmats, d_tiles, iter, sc, s,
-                                                        device_status_ptr());
+    if (sc.bf16_mode) return cudaErrorInvalidValue;   // fp32 mode only: its workspace holds fp32 X, A and B
+    simt_phase_kernel<<<ntiles, 256, 0, st>>>(ph, d_mats, nmats, d_tiles, iter, sc, s, device_status_ptr());
     return cudaGetLastError();
 }
 

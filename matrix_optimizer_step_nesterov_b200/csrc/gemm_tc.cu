@@ -26,7 +26,11 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
+#include <functional>
 #include <mutex>
+#include <queue>
+#include <utility>
 #include <vector>
 
 namespace mfsdp {
@@ -523,10 +527,13 @@ constexpr bool kSymA = ph == PH_POLY || ph == PH_APPLY || ph == PH_FINAL;
 template <int ph>
 constexpr bool kSymB = ph == PH_POLY;
 
+// Tiles come from a host-built table partitioned per cluster: cluster k runs
+// tiles[seg[k]] .. tiles[seg[k + 1] - 1] in that order (every role of both
+// CTAs walks the same segment).
 template <int ph, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps, int32_t nmats,
-                const TileDev* __restrict__ tiles, int32_t ntiles, int32_t iter, StepScalars sc,
+                const TileDev* __restrict__ tiles, const int32_t* __restrict__ seg, int32_t iter, StepScalars sc,
                 const float* __restrict__ s, int32_t* status) {
     using C = TcCfg<CG>;
     constexpr int STAGES = C::STAGES;
@@ -546,7 +553,8 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
     const uint32_t mma_done = smem_u32(bars + 2 * STAGES + 4);
     const uint32_t rank = (CG == 2) ? cluster_rank() : 0u;      // 0 = leader (issues the MMAs)
     const bool leader = rank == 0;
-    const int cluster_id = blockIdx.x / CG, nclusters = gridDim.x / CG;
+    const int cluster_id = blockIdx.x / CG;
+    const int t_begin = seg[cluster_id], t_end = seg[cluster_id + 1];
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -590,7 +598,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             int issued[STAGES];                  // parity of the last fill issued per stage, -1 = none
             #pragma unroll
             for (int i = 0; i < STAGES; ++i) issued[i] = -1;
-            for (int t = cluster_id; t < ntiles && ok; t += nclusters) {
+            for (int t = t_begin; t < t_end && ok; ++t) {
                 const TileDev td = tiles[t];
                 const MatDev& md = mats[td.mat];
                 const TcMaps& mp = maps[td.mat];
@@ -655,7 +663,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = cluster_id; t < ntiles && ok; t += nclusters) {
+            for (int t = t_begin; t < t_end && ok; ++t) {
                 const TileDev td = tiles[t];
                 const MatDev& md = mats[td.mat];
                 const int K = (ph == PH_GRAM) ? md.c : md.r;
@@ -708,7 +716,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
         const uint32_t tempty_leader0 = (CG == 2) ? map_to_rank(tempty0, 0) : tempty0;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = cluster_id; t < ntiles; t += nclusters) {
+        for (int t = t_begin; t < t_end; ++t) {
             const TileDev td = tiles[t];
             const MatDev md = mats[td.mat];   // a register copy: global stores below cannot alias it
             const int Mrows = md.r;
@@ -829,8 +837,6 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 
 }  // namespace
 
-bool tc_available() { return true; }
-
 cudaError_t launch_bounded_wait_selftest(unsigned long long limit_ns, cudaStream_t st) {
     bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, device_status_ptr());
     return cudaGetLastError();
@@ -858,8 +864,43 @@ bool tc_encode_maps(const std::vector<MatDev>& mats, void* host_out) {
     return true;
 }
 
-void tc_build_tiles(const std::vector<MatDev>& mats, std::vector<TileDev>& gram, std::vector<TileDev>& poly,
-                    std::vector<TileDev>& gen) {
+namespace {
+
+// Longest-processing-time assignment of a sorted tile list to nclusters
+// clusters: each tile goes to the cluster with the least work so far (lowest
+// id on ties), and every cluster keeps its tiles in list order.  A tile's
+// work is its K depth in 64-deep blocks, but at least the epilogue's cost
+// in the same units (the epilogue of one tile overlaps the next tile's MMAs,
+// so a short tile still costs about one epilogue), plus one block of fixed
+// overhead.  The list is rewritten cluster by cluster and seg gets the
+// nclusters + 1 segment offsets.
+void partition_lpt(std::vector<TileDev>& tiles, int nclusters, int epi_blocks, std::vector<int32_t>& seg) {
+    nclusters = std::max(1, nclusters);
+    std::vector<std::vector<TileDev>> per(static_cast<size_t>(nclusters));
+    using Load = std::pair<int64_t, int>;
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int c = 0; c < nclusters; ++c) heap.push({0, c});
+    for (const TileDev& t : tiles) {
+        const Load l = heap.top();
+        heap.pop();
+        per[l.second].push_back(t);
+        heap.push({l.first + std::max(t.kblk, epi_blocks) + 1, l.second});
+    }
+    seg.assign(static_cast<size_t>(nclusters) + 1, 0);
+    tiles.clear();
+    for (int c = 0; c < nclusters; ++c) {
+        tiles.insert(tiles.end(), per[c].begin(), per[c].end());
+        seg[c + 1] = static_cast<int32_t>(tiles.size());
+    }
+}
+
+}  // namespace
+
+int tc_launch_clusters(int ntiles, int max_clusters) { return std::max(1, std::min(ntiles, max_clusters)); }
+
+void tc_build_tiles(const std::vector<MatDev>& mats, int max_clusters, std::vector<TileDev>& gram,
+                    std::vector<TileDev>& poly, std::vector<TileDev>& gen, std::vector<int32_t>& gram_seg,
+                    std::vector<int32_t>& poly_seg, std::vector<int32_t>& gen_seg) {
     constexpr int TM = TcCfg<kCtaGroup>::TILE_M;
     for (int32_t mi = 0; mi < static_cast<int32_t>(mats.size()); ++mi) {
         const MatDev& m = mats[mi];
@@ -894,68 +935,106 @@ void tc_build_tiles(const std::vector<MatDev>& mats, std::vector<TileDev>& gram,
     std::stable_sort(gram.begin(), gram.end(), lpt);
     std::stable_sort(poly.begin(), poly.end(), lpt);
     std::stable_sort(gen.begin(), gen.end(), lpt_cols);
+    // epilogue cost per tile in K blocks (measured order of magnitude): GRAM
+    // stores one bf16 tile, POLY also reads one, APPLY reads and writes X's
+    // two bf16 parts
+    partition_lpt(gram, tc_launch_clusters(static_cast<int>(gram.size()), max_clusters), 4, gram_seg);
+    partition_lpt(poly, tc_launch_clusters(static_cast<int>(poly.size()), max_clusters), 6, poly_seg);
+    partition_lpt(gen, tc_launch_clusters(static_cast<int>(gen.size()), max_clusters), 10, gen_seg);
 }
 
 namespace {
 
-template <int ph>
-cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats, const TileDev* d_tiles,
-                         int32_t ntiles, int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st,
-                         int sms) {
+constexpr int kMaxDevices = 64;
+
+cudaLaunchConfig_t phase_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr) {
     constexpr int CG = kCtaGroup;
-    // one-time, thread-safe set-up of this phase's kernel
-    static const cudaError_t attr_err = cudaFuncSetAttribute(
-        tc_phase_kernel<ph, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<CG>::SMEM_BYTES);
-    if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((sms / CG) * CG, 1, 1);
+    cfg.gridDim = dim3(clusters * CG, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = TcCfg<CG>::SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CG;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // clusters of CG CTAs that fit on the device at once (computed once)
-    static const int max_clusters = [&] {
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, tc_phase_kernel<ph, CG>, &cfg) != cudaSuccess || n <= 0) {
-            cudaGetLastError();
-            n = sms / CG;
-        }
-        return n;
-    }();
-    const int clusters = std::max(1, std::min(ntiles, max_clusters));
-    cfg.gridDim = dim3(clusters * CG, 1, 1);
-    return cudaLaunchKernelEx(&cfg, tc_phase_kernel<ph, CG>, d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s,
+    return cfg;
+}
+
+// Per device, once: the phase kernels' shared-memory attribute, then the
+// number of CTA-pair clusters that fit on the device at once (the persistent
+// grid).  0 on error.
+int device_clusters() {
+    static std::atomic<int> cached[kMaxDevices];   // zero-initialised: unknown
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 0;
+    }
+    int n = cached[dev].load(std::memory_order_acquire);
+    if (n > 0) return n;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    n = cached[dev].load(std::memory_order_acquire);
+    if (n > 0) return n;
+    constexpr int CG = kCtaGroup;
+    const int smem = TcCfg<CG>::SMEM_BYTES;
+    if (cudaFuncSetAttribute(tc_phase_kernel<PH_GRAM, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(tc_phase_kernel<PH_POLY, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(tc_phase_kernel<PH_APPLY, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(tc_phase_kernel<PH_FINAL, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        return 0;
+    }
+    // the four phase kernels share one launch shape (threads, shared memory, cluster)
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = phase_config(sms / CG, nullptr, attr);
+    if (cudaOccupancyMaxActiveClusters(&n, tc_phase_kernel<PH_APPLY, CG>, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = sms / CG;
+    }
+    cached[dev].store(n, std::memory_order_release);
+    return n;
+}
+
+template <int ph>
+cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats, const TileDev* d_tiles,
+                         const int32_t* d_seg, int32_t clusters, int32_t iter, const StepScalars& sc, const float* s,
+                         cudaStream_t st) {
+    constexpr int CG = kCtaGroup;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = phase_config(clusters, st, attr);
+    return cudaLaunchKernelEx(&cfg, tc_phase_kernel<ph, CG>, d_mats, maps, nmats, d_tiles, d_seg, iter, sc, s,
                               device_status_ptr());
 }
 
 }  // namespace
 
+int tc_max_clusters() { return device_clusters(); }
+
 cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, int32_t nmats,
-                           const TileDev* d_tiles, int32_t ntiles, int32_t iter, const StepScalars& sc,
-                           const float* s, cudaStream_t st) {
-    if (ntiles <= 0) return cudaSuccess;
-    static const int sms = [] {
-        int dev = 0, c = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) {
-            cudaGetLastError();
-            c = 148;
-        }
-        return c;
-    }();
+                           const TileDev* d_tiles, const int32_t* d_seg, int32_t clusters, int32_t iter,
+                           const StepScalars& sc, const float* s, cudaStream_t st) {
+    if (clusters <= 0) return cudaSuccess;
+    if (device_clusters() <= 0) return cudaErrorInvalidConfiguration;   // attributes not set on this device
     const TcMaps* maps = static_cast<const TcMaps*>(d_maps);
     cudaError_t e;
     switch (ph) {
-        case PH_GRAM: e = launch_phase<PH_GRAM>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, st, sms); break;
-        case PH_POLY: e = launch_phase<PH_POLY>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, st, sms); break;
-        case PH_APPLY: e = launch_phase<PH_APPLY>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, st, sms); break;
-        default: e = launch_phase<PH_FINAL>(d_mats, maps, nmats, d_tiles, ntiles, iter, sc, s, st, sms); break;
+        case PH_GRAM: e = launch_phase<PH_GRAM>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, sc, s, st); break;
+        case PH_POLY: e = launch_phase<PH_POLY>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, sc, s, st); break;
+        case PH_APPLY: e = launch_phase<PH_APPLY>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, sc, s, st); break;
+        default: e = launch_phase<PH_FINAL>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, sc, s, st); break;
     }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
