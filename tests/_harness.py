@@ -2,7 +2,7 @@
 
 The two sides share only the seeded inputs from ``synth``.  The GPU side goes
 through ``matrix_optimizer_step_nesterov_b200`` (libmfsdp); the oracle side
-through ``oracle``.  No expected value is ever taken from the GPU path except
+through ``oracle`` (its fp64 C++ library).  No expected value is ever taken from the GPU path except
 where a check is explicitly "given the GPU's own O" (the parameter-write
 check, which tests the write alone).
 """
@@ -79,12 +79,15 @@ class GpuResult:
 
 def gpu_step(hs: HostState, mode: str, want_o: Optional[Sequence[int]] = None, ns_steps: int = 5,
              nesterov: bool = True, lr: float = 0.02, beta: float = 0.95, weight_decay: float = 0.01,
-             grads: Optional[List[np.ndarray]] = None, repeat: int = 1) -> GpuResult:
+             grads: Optional[List[np.ndarray]] = None, repeat: int = 1, keep: Optional[Sequence[int]] = None
+             ) -> GpuResult:
     """Run the product step over every matrix of ``hs`` in ONE grouped call
-    (``repeat`` calls in a row with the same gradients)."""
+    (``repeat`` calls in a row with the same gradients).  ``keep`` limits the
+    matrices whose W and momentum are copied back (default: all)."""
     from matrix_optimizer_step_nesterov_b200 import MuonOwnerStep
     dev = torch.device("cuda")
     want = set(range(len(hs.specs))) if want_o is None else set(want_o)
+    kept = set(range(len(hs.specs))) if keep is None else set(keep)
     params, gs, bufs, outs = [], [], [], []
     for k, s in enumerate(hs.specs):
         dt = _TORCH_DT[s.dtype]
@@ -98,9 +101,9 @@ def gpu_step(hs: HostState, mode: str, want_o: Optional[Sequence[int]] = None, n
     for _ in range(repeat):
         step.step()
     torch.cuda.synchronize()
-    res = GpuResult([p.cpu() for p in params],
+    res = GpuResult([p.cpu() if k in kept else None for k, p in enumerate(params)],
                     [o.cpu().numpy().astype(np.float64) if o is not None else None for o in outs],
-                    [b.cpu().numpy() for b in bufs])
+                    [b.cpu().numpy() if k in kept else None for k, b in enumerate(bufs)])
     step.close()
     del params, gs, bufs, outs
     return res
@@ -157,8 +160,10 @@ def check_write(W0: np.ndarray, O_gpu: np.ndarray, W_gpu: torch.Tensor, lr: floa
     return {"write_ulp": ulp, "write_excess": excess}
 
 
-def compare_matrix(hs: HostState, res: GpuResult, k: int, mode: str, **kw) -> Dict[str, float]:
-    Wn, O, bn = oracle_step(hs, k, **kw)
+def compare_matrix(hs: HostState, res: GpuResult, k: int, mode: str, ref=None, **kw) -> Dict[str, float]:
+    """Errors of matrix k of a GPU result against the oracle on the same inputs
+    (``ref`` = a precomputed oracle_step(hs, k, **kw), else computed here)."""
+    Wn, O, bn = ref if ref is not None else oracle_step(hs, k, **kw)
     out = {"rel_O": rel_frob(res.O[k], O) if res.O[k] is not None else float("nan"),
            "rel_buf": rel_frob(res.buf[k], bn)}
     if res.O[k] is not None:

@@ -69,10 +69,8 @@ def test_p2p_step_parity_and_copies(mode):
     st.close()
     hp = H.muon_hparams_as_passed()
     for k in range(len(shapes)):
-        G = np.zeros(shapes[k], np.float64)
-        for p in parts[k]:
-            G += p.astype(np.float64)
-        Wn, On, bn = oracle.muon_step(hs.W[k], G, hs.buf[k], hp)
+        # the oracle's owner-segment form: the ranks' contributions summed in rank order
+        Wn, On, bn = oracle.muon_step_parts(hs.W[k], parts[k], hs.buf[k], hp)
         assert H.rel_frob(O[k].cpu().numpy(), On) <= H.TOL_O[mode]
         assert H.rel_frob(B[k].cpu().numpy(), bn) <= H.TOL_BUF
         for c in C[k]:
