@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "owner-step latency (ms) & NS5 TFLOP/s at 7B owner share; tail AdamW GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_HBM_GBS = 8000.0      # B200 HBM3e, the nominal figure (for a second fraction beside the measured one)
 
 
 # ---- host-side logic shared with the CPU tests --------------------------------------
@@ -56,6 +57,19 @@ def product_plan(params, world_size):
 def product_heaviest(F, B):
     from matrix_optimizer_step_nesterov_b200 import mfsdp_heaviest_rank
     return mfsdp_heaviest_rank(F, B)
+
+
+def plan_balance(params, world_size: int) -> dict:
+    """Balance of the owner plan over ``world_size`` ranks (host only): the
+    heaviest rank's Newton-Schulz FLOPs and resident bytes over the per-rank
+    means.  A multi-GPU step's makespan is the heaviest rank's step."""
+    shards, F, B = product_plan(params, world_size)
+    h = product_heaviest(F, B)
+    mf, mb = sum(F) / len(F), sum(B) / len(B)
+    return {"world_size": world_size, "heaviest_rank": h,
+            "imbalance_flops": round(max(F) / mf, 6) if mf > 0 else None,
+            "imbalance_bytes": round(max(B) / mb, 6) if mb > 0 else None,
+            "ranks_with_matrices": sum(1 for f in F if f > 0)}
 
 
 def ns_flops_algorithmic(specs, steps: int = 5) -> float:
@@ -217,53 +231,68 @@ def gpu_index_of(dev: int) -> Optional[str]:
 
 # ---- oracle timing (cpu baseline / reference arm) ---------------------------------------------
 
-def blas_threads() -> int:
-    try:
-        import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        return max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=1)
-    except Exception:
-        return os.cpu_count() or 1
+def oracle_threads() -> int:
+    import oracle
+    return oracle.native.threads()
 
 
-def oracle_share_estimate(wl, specs, tail_n: int, budget_s: float = 20.0, one_shape: bool = False):
-    """Time the fp64 oracle on one matrix per distinct shape (ascending FLOPs, until
-    ``budget_s``), extrapolate unmeasured shapes by the measured FLOP rate, scale
-    by shape counts, and add AdamW over the whole tail.  Returns (ms, sample text)."""
+def oracle_share_estimate(wl, specs, tail_n: int, budget_s: float = 20.0):
+    """Host time of the fp64 C++ oracle on the owner's whole step, from a bounded sample.
+
+    The oracle's step on one matrix is momentum + norm + write (the same work
+    whatever ns_steps is) plus ns_steps identical Newton-Schulz iterations, so
+    its time is T(ns) = T(0) + ns (T(1) - T(0)).  For each distinct shape, in
+    ascending size until ``budget_s`` is spent, one matrix is timed at ns = 0
+    and ns = 1 and its full-step time taken from that line; shapes past the
+    budget are extrapolated at the measured rate of dense Newton-Schulz FLOPs
+    per second.  The per-shape times are scaled by the shape counts, and AdamW
+    over the whole tail is added (timed whole).  Both benchmark arms use this
+    one estimator.  Returns a dict: ms, sample text, seconds of oracle work
+    measured, extrapolation factor (estimated / measured oracle seconds)."""
+    import dataclasses
     import oracle
     from synth.gen import matrix_inputs, tail_inputs
     by_shape: Dict[tuple, list] = {}
     for s in specs:
         by_shape.setdefault((s.rows, s.cols), []).append(s)
     shapes = sorted(by_shape, key=lambda sh: ns_flops_dense([by_shape[sh][0]]))
-    hp = oracle.MuonHParams()
-    measured = {}
+    hp5 = oracle.MuonHParams()
+    per_shape = {}
     spent = 0.0
     for sh in shapes:
-        if measured and (spent > budget_s or one_shape):
+        if per_shape and spent > budget_s:
             break
         mi = matrix_inputs(wl, by_shape[sh][0])
-        t0 = time.perf_counter()
-        oracle.muon_step(mi.W, mi.G, mi.buf, hp)
-        dt = time.perf_counter() - t0
-        measured[sh] = dt
-        spent += dt
-    rate = sum(ns_flops_dense([by_shape[sh][0]]) for sh in measured) / sum(measured.values())
+        t = []
+        for ns in (0, 1):
+            t0 = time.perf_counter()
+            oracle.muon_step(mi.W, mi.G, mi.buf, dataclasses.replace(hp5, ns_steps=ns))
+            t.append(time.perf_counter() - t0)
+        spent += t[0] + t[1]
+        per_shape[sh] = (t[0], t[1], t[0] + hp5.ns_steps * max(t[1] - t[0], 0.0))
+    measured_flops = sum(ns_flops_dense([by_shape[sh][0]], steps=1) for sh in per_shape)
+    rate = measured_flops / max(sum(v[1] - v[0] for v in per_shape.values()), 1e-9)
     total = 0.0
     for sh in shapes:
-        per = measured.get(sh, ns_flops_dense([by_shape[sh][0]]) / rate)
-        total += per * len(by_shape[sh])
-    tail_ms = 0.0
+        full = per_shape[sh][2] if sh in per_shape else ns_flops_dense([by_shape[sh][0]]) / rate
+        total += full * len(by_shape[sh])
+    tail_s = 0.0
     if tail_n:
         ti = tail_inputs(wl)
         t0 = time.perf_counter()
         oracle.adamw_step(ti.p, ti.g, ti.m, ti.v, 1, oracle.AdamWHParams())
-        tail_ms = (time.perf_counter() - t0) * 1e3
-    sample = (f"oracle muon_step on one matrix of each of {len(measured)}/{len(shapes)} distinct shapes "
-              f"({', '.join(f'{r}x{c}' for r, c in measured)}), other shapes extrapolated at the measured "
-              f"fp64 rate {rate / 1e9:.1f} GFLOP/s, scaled by shape counts over {len(specs)} matrices; "
-              f"AdamW over the whole {tail_n}-element tail")
-    return total * 1e3 + tail_ms, sample, spent
+        tail_s = time.perf_counter() - t0
+        spent += tail_s
+    est_s = total + tail_s
+    sample = (f"fp64 C++ oracle on {oracle_threads()} host threads: one matrix of each of {len(per_shape)}/"
+              f"{len(shapes)} distinct shapes ({', '.join(f'{r}x{c}' for r, c in per_shape)}) timed at "
+              f"ns_steps = 0 and 1, full step = T(0) + {hp5.ns_steps} (T(1) - T(0))"
+              + (f", other shapes at the measured {rate / 1e9:.1f} GFLOP/s" if len(per_shape) < len(shapes) else "")
+              + f", scaled by shape counts over {len(specs)} matrices; AdamW timed over the whole "
+              f"{tail_n}-element tail; value extrapolated x{est_s / max(spent, 1e-9):.1f} from {spent:.1f} s "
+              "of measured oracle work")
+    return {"ms": est_s * 1e3, "sample": sample, "spent_s": spent,
+            "extrapolation": est_s / max(spent, 1e-9), "gflops": rate / 1e9}
 
 
 # ---- the GPU arm --------------------------------------------------------------------------------------
@@ -294,6 +323,7 @@ def run_ours(args) -> int:
     else:
         planned, specs, owns_tail, _ = planned_share(wl.params, R, rank, product_plan, product_heaviest)
     tail_n = wl.tail_numel if owns_tail else 0
+    plan_info = plan_balance(wl.params, R) if wl.world_size else None
 
     t_gen = time.perf_counter()
     ins = matrix_inputs_many(wl, specs)
@@ -487,7 +517,8 @@ def run_ours(args) -> int:
                 # 2 x 4096^2 + 4096x11008 + 11008x4096, scaled to the 7B share (GRAM and APPLY by X's
                 # elements, POLY by A's) and averaged over a step's 15 GEMM launches
                 "traffic": GEMM_TRAFFIC_7B if wl.name == "7b_share" else None,
-                "traffic_note": "scaled from a 4-matrix capture (profiles/tc_phase_kernel_4x4096.md)"
+                "traffic_note": "ncu DRAM bytes of one GRAM, POLY and APPLY launch on four 7B-share matrices, "
+                                "scaled to the share and averaged over a step's GEMM launches"
                                 if wl.name == "7b_share" else None,
                 "kernel": "Newton-Schulz GEMM phases (gram + poly + apply + final launches)",
                 "flops_per_launch": flops_alg * steps_timed / max(gemm_launches, 1),
@@ -509,21 +540,35 @@ def run_ours(args) -> int:
     if tail_bench:
         tail_roof = {"bound": "hbm", "achieved": tail_bench["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(tail_bench["gbs"] / peaks["hbm_gbs"], 4),
+                     "frac_of_spec": round(tail_bench["gbs"] / SPEC_HBM_GBS, 4),
                      # ncu dram__bytes_read.sum + dram__bytes_write.sum of one 64 Mi launch
                      "traffic": 1.8233e9 if tail_bench["elements"] == 64 << 20 else None,
                      "kernel": "AdamW tail, 64 Mi fp32 elements, 28 B/elem"}
-    mom = prof.get("momentum")
-    mom_gbs = None
-    if mom and mom[1] > 0:
+    # the streaming kernels of the matrix step, from the same timed region
+    n_elems = sum(s.numel for s in specs)
+    wbytes = 2 if all(s.dtype == "bf16" for s in specs) else 4
+    hbm_kernels = {
         # bf16 mode: G 2 + buf 4 in, buf 4 + X hi 2 + X lo 2 out; fp32 mode: G 4 + buf 4 in, buf 4 + X 4 out
-        mom_bytes = sum(s.numel for s in specs) * (14 if args.mode == "bf16" else 16)
-        mom_gbs = round(mom_bytes * mom[0] / (mom[1] * 1e-3) / 1e9, 1)
+        "momentum": n_elems * (14 if args.mode == "bf16" else 16),
+        # bf16 mode: X hi 2 + X lo 2 + W in, W out; fp32 mode: X 4 + W in, W out
+        "write": n_elems * (4 + 2 * wbytes),
+    }
+    roof_hbm = {}
+    for k, nbytes in hbm_kernels.items():
+        v = prof.get(k)
+        if v and v[1] > 0:
+            gbs = nbytes * v[0] / (v[1] * 1e-3) / 1e9
+            roof_hbm[k] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": round(gbs / peaks["hbm_gbs"], 4), "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4),
+                           "bytes_per_launch": nbytes, "avg_launch_ms": round(v[1] / v[0], 5)}
+    mom_gbs = roof_hbm.get("momentum", {}).get("achieved")
 
     cpu_baseline = None
     if world == 1 and not args.no_cpu_baseline:
-        est_ms, sample, spent = oracle_share_estimate(wl, specs, tail_n, budget_s=args.cpu_budget)
-        cpu_baseline = {"value": round(est_ms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
-                        "sample": sample, "cpu_seconds_spent": round(spent, 1)}
+        est = oracle_share_estimate(wl, specs, tail_n, budget_s=args.cpu_budget)
+        cpu_baseline = {"value": round(est["ms"], 1), "unit": "ms", "cores": oracle_threads(), "kind": "oracle",
+                        "sample": est["sample"], "cpu_seconds_spent": round(est["spent_s"], 1),
+                        "extrapolation": round(est["extrapolation"], 2)}
 
     line = {
         "metric": METRIC,
@@ -556,6 +601,8 @@ def run_ours(args) -> int:
         "momentum_gbs": mom_gbs,
         "roofline": roof,
         "roofline_tail": tail_roof,
+        "roofline_hbm": roof_hbm or None,
+        "plan": plan_info,
         "phases": phases,
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
@@ -573,10 +620,12 @@ def run_ours(args) -> int:
 # ---- the reference arm: the oracle on host cores -------------------------------------------------------
 
 def run_reference(args) -> int:
+    """The reference arm: the fp64 C++ oracle on the host cores, as it stands.
+    Each step runs the same bounded-sample estimator as the GPU arm's
+    cpu_baseline leg; warm-up steps run it on the smallest shape only."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    from synth import workload
     import oracle
     wl = bench_workload(args)
     R = wl.world_size or 1
@@ -585,21 +634,22 @@ def run_reference(args) -> int:
     else:
         _, specs, owns_tail, _ = planned_share(wl.params, R, 0, oracle.plan_owners, oracle.heaviest_rank)
     tail_n = wl.tail_numel if owns_tail else 0
-    vals = []
-    sample = ""
-    for k in range(args.warmup + args.steps):
-        est, sample, _ = oracle_share_estimate(wl, specs, tail_n, one_shape=True)
-        if k >= args.warmup:
-            vals.append(est)
-    v = statistics.mean(vals)
+    smallest = [min(specs, key=lambda s: ns_flops_dense([s]))]
+    for _ in range(args.warmup):
+        oracle_share_estimate(wl, smallest, 0, budget_s=0.0)
+    ests = [oracle_share_estimate(wl, specs, tail_n, budget_s=args.cpu_budget) for _ in range(args.steps)]
+    v = statistics.median(e["ms"] for e in ests)
+    spent = sum(e["spent_s"] for e in ests)
     line = {
         "impl": "reference",
         "metric": METRIC, "value": round(v, 1), "unit": "ms", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 1), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{wl.name}: {wl.description}", "matrices": len(specs), "tail_elements": tail_n},
-        "cpu_baseline": {"value": round(v, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
-                         "sample": "each step: " + sample},
+        "cpu_baseline": {"value": round(v, 1), "unit": "ms", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": "each step (median of the steps): " + ests[-1]["sample"],
+                         "cpu_seconds_spent": round(spent, 1),
+                         "extrapolation": round(statistics.median(e["extrapolation"] for e in ests), 2)},
         "e2e": {"value": round(v, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -621,7 +671,8 @@ def main(argv=None) -> int:
     ap.add_argument("--e2e-groups", type=int, default=6, help="matrix groups pipelined in the e2e measurement")
     ap.add_argument("--no-tail-bench", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle work after which unmeasured shapes are extrapolated")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
