@@ -211,9 +211,11 @@ int mfsdp_muon_workspace_size(const mfsdp_matrix* mats, int32_t n, const mfsdp_m
  *   stream           cudaStream_t as void*
  * Alignment: param/grad aligned to their element size, momentum and
  * update_out to 4 bytes (16-byte alignment enables vector access).  Matrices
- * must not alias one another.  Launches: one momentum kernel, one norm kernel,
- * three GEMM-phase kernels per Newton-Schulz iteration, one parameter-write
- * kernel.
+ * must not alias one another.  Launches: the momentum kernel and the
+ * parameter-write kernel once each for the flat matrices (untransposed, rows a
+ * multiple of 8 elements, every buffer 16-byte aligned) and once each for the
+ * others, one norm kernel, three GEMM-phase kernels per Newton-Schulz
+ * iteration (mfsdp_muon_step_launches counts them).
  * Errors: MFSDP_ERR_INVALID_ARG, MFSDP_ERR_UNSUPPORTED_DTYPE, MFSDP_ERR_MISALIGNED,
  * MFSDP_ERR_WORKSPACE_TOO_SMALL, MFSDP_ERR_UNSUPPORTED_DEVICE, MFSDP_ERR_CUDA.
  */
@@ -262,12 +264,45 @@ int mfsdp_muon_workspace_size_p2p(const mfsdp_matrix* mats, const mfsdp_owner_se
 int mfsdp_muon_step_p2p(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
                         const mfsdp_muon_hparams* hp, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- owner-segment materialisation overlapped with the step ---------------
+ * Passage: the same as mfsdp_muon_step_p2p (gist.science French summary,
+ * Methodologie section 2, "Collectifs P2P Segment-Proprietaire": the owner
+ * materialises its updated segments to the ranks that need them).  The step of
+ * mfsdp_muon_step_p2p, split into `groups` contiguous groups of the list (in
+ * list order, of about equal Newton-Schulz work), stepped one after another on
+ * `stream`; as soon as a group's parameters are written, their copies to every
+ * param_copies[d] are enqueued on `copy_stream` and run on the copy engines
+ * while the later groups compute.  Before returning, the call makes `stream`
+ * wait for every copy, so work enqueued on `stream` afterwards sees all of them.
+ *   groups       1..64 (1: no overlap, the copies follow the whole step)
+ *   copy_stream  cudaStream_t as void*, a stream other than `stream` for the
+ *                overlap (NULL = the legacy default stream, which serialises)
+ *   workspace    >= mfsdp_muon_workspace_size_p2p_overlap() bytes, 256-byte
+ *                aligned: one region per group, each with the workspace rules of
+ *                mfsdp_muon_step; call mfsdp_muon_forget_workspace_range() on the
+ *                whole workspace before giving the memory another use
+ * Results are bit for bit those of mfsdp_muon_step_p2p with the same arguments.
+ * Errors: those of mfsdp_muon_step_p2p.
+ */
+int mfsdp_muon_workspace_size_p2p_overlap(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                                          const mfsdp_muon_hparams* hp, int32_t groups, size_t* bytes);
+
+int mfsdp_muon_step_p2p_overlap(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                                const mfsdp_muon_hparams* hp, int32_t groups, void* workspace,
+                                size_t workspace_bytes, void* stream, void* copy_stream);
+
 /* Number of kernel launches one mfsdp_muon_step call with these arguments enqueues. */
 int mfsdp_muon_step_launches(const mfsdp_matrix* mats, int32_t n, const mfsdp_muon_hparams* hp,
                              int32_t* launches);
 
 /* Drop the host-side cache entry for a workspace (before reusing its memory). */
 int mfsdp_muon_forget_workspace(void* workspace);
+
+/* Drop every host-side cache entry for workspaces that start inside
+ * [workspace, workspace + bytes): the per-group regions of a
+ * mfsdp_muon_step_p2p_overlap workspace.  Errors: MFSDP_ERR_INVALID_ARG
+ * (the range wraps around). */
+int mfsdp_muon_forget_workspace_range(void* workspace, size_t bytes);
 
 /*
  * mfsdp_muon_step_noalloc - mfsdp_muon_step without a caller workspace, for

@@ -39,7 +39,8 @@ EXPORTED = (
     "mfsdp_get_device_status", "mfsdp_status_string", "mfsdp_version",
     "mfsdp_profile_begin", "mfsdp_profile_end", "mfsdp_muon_step_noalloc",
     "mfsdp_muon_workspace_size_p2p", "mfsdp_muon_step_p2p", "mfsdp_selftest_bounded_wait",
-    "mfsdp_reshard",
+    "mfsdp_reshard", "mfsdp_muon_workspace_size_p2p_overlap", "mfsdp_muon_step_p2p_overlap",
+    "mfsdp_muon_forget_workspace_range",
 )
 
 MFSDP_MAX_PARTS = 64
@@ -134,6 +135,8 @@ def load() -> ctypes.CDLL:
     lib.mfsdp_muon_step_launches.restype = ctypes.c_int
     lib.mfsdp_muon_forget_workspace.argtypes = [p]
     lib.mfsdp_muon_forget_workspace.restype = ctypes.c_int
+    lib.mfsdp_muon_forget_workspace_range.argtypes = [p, ctypes.c_size_t]
+    lib.mfsdp_muon_forget_workspace_range.restype = ctypes.c_int
     lib.mfsdp_adamw_tail.argtypes = [p, p, p, p, i64, ctypes.POINTER(AdamWHParams), p]
     lib.mfsdp_adamw_tail.restype = ctypes.c_int
     lib.mfsdp_get_device_status.argtypes = [p, ctypes.POINTER(ctypes.c_int32)]
@@ -150,6 +153,13 @@ def load() -> ctypes.CDLL:
     lib.mfsdp_muon_step_p2p.argtypes = [ctypes.POINTER(Matrix), ctypes.POINTER(OwnerSegments), i32,
                                         ctypes.POINTER(MuonHParams), p, ctypes.c_size_t, p]
     lib.mfsdp_muon_step_p2p.restype = ctypes.c_int
+    lib.mfsdp_muon_workspace_size_p2p_overlap.argtypes = [ctypes.POINTER(Matrix), ctypes.POINTER(OwnerSegments),
+                                                          i32, ctypes.POINTER(MuonHParams), i32,
+                                                          ctypes.POINTER(ctypes.c_size_t)]
+    lib.mfsdp_muon_workspace_size_p2p_overlap.restype = ctypes.c_int
+    lib.mfsdp_muon_step_p2p_overlap.argtypes = [ctypes.POINTER(Matrix), ctypes.POINTER(OwnerSegments), i32,
+                                                ctypes.POINTER(MuonHParams), i32, p, ctypes.c_size_t, p, p]
+    lib.mfsdp_muon_step_p2p_overlap.restype = ctypes.c_int
     lib.mfsdp_muon_step_noalloc.argtypes = [ctypes.POINTER(Matrix), i32, ctypes.POINTER(MuonHParams), p]
     lib.mfsdp_muon_step_noalloc.restype = ctypes.c_int
     lib.mfsdp_selftest_bounded_wait.argtypes = [i64, p]
@@ -254,6 +264,10 @@ def mfsdp_muon_forget_workspace(workspace_ptr: int) -> None:
     _check(load().mfsdp_muon_forget_workspace(workspace_ptr), "mfsdp_muon_forget_workspace")
 
 
+def mfsdp_muon_forget_workspace_range(workspace_ptr: int, nbytes: int) -> None:
+    _check(load().mfsdp_muon_forget_workspace_range(workspace_ptr, nbytes), "mfsdp_muon_forget_workspace_range")
+
+
 # ---- AdamW tail ------------------------------------------------------------------
 
 def adamw_hparams(lr=0.02, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.01, step=1) -> AdamWHParams:
@@ -338,3 +352,20 @@ def mfsdp_muon_step_p2p(mats: Sequence[Matrix], segs, hp: MuonHParams, workspace
         arr = matrix_array(mats)
     _check(load().mfsdp_muon_step_p2p(arr, segs, len(mats), ctypes.byref(hp), workspace_ptr, workspace_bytes,
                                       stream), "mfsdp_muon_step_p2p")
+
+
+def mfsdp_muon_workspace_size_p2p_overlap(mats: Sequence[Matrix], segs, hp: MuonHParams, groups: int) -> int:
+    out = ctypes.c_size_t()
+    _check(load().mfsdp_muon_workspace_size_p2p_overlap(matrix_array(mats), segs, len(mats), ctypes.byref(hp),
+                                                        int(groups), ctypes.byref(out)),
+           "mfsdp_muon_workspace_size_p2p_overlap")
+    return out.value
+
+
+def mfsdp_muon_step_p2p_overlap(mats: Sequence[Matrix], segs, hp: MuonHParams, groups: int, workspace_ptr: int,
+                                workspace_bytes: int, stream: int, copy_stream: int, arr=None) -> None:
+    if arr is None:
+        arr = matrix_array(mats)
+    _check(load().mfsdp_muon_step_p2p_overlap(arr, segs, len(mats), ctypes.byref(hp), int(groups), workspace_ptr,
+                                              workspace_bytes, stream, copy_stream),
+           "mfsdp_muon_step_p2p_overlap")

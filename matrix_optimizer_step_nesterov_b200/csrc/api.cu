@@ -21,6 +21,7 @@ namespace mfsdp {
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr size_t kRegionSlack = 128;
 
 size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
@@ -141,7 +142,8 @@ struct Layout {
     std::vector<uint64_t> ptrs;        // owner-segment part and copy pointers, per matrix
     size_t off_ptrs = 0;
     int32_t mom_tiles = 0;
-    int32_t mom_groups = 0;
+    int32_t mom_groups = 0;            // groups of the streaming kernels, flat ones first
+    int32_t flat_groups = 0;           // groups of the flat matrices: [0, flat_groups)
     size_t off_mats = 0, off_maps = 0, off_sym = 0, off_poly = 0, off_gen = 0, off_partials = 0, off_s = 0;
     size_t off_sym_seg = 0, off_poly_seg = 0, off_gen_seg = 0;
     size_t head_end = 0, maps_bytes = 0;
@@ -240,7 +242,7 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
         const mfsdp_matrix& u = in[i];
         if (u.rows == 0 || u.cols == 0) continue;
         MatDev m{};
-        bool vec_parts = true;
+        bool vec_parts = true, vec_parts16 = true;
         if (segs) {
             const mfsdp_owner_segments& sg = segs[i];
             m.nparts = sg.nparts;
@@ -249,6 +251,7 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
             for (int32_t r = 0; r < sg.nparts; ++r) {
                 L.ptrs.push_back(reinterpret_cast<uint64_t>(sg.grad_parts[r]));
                 vec_parts = vec_parts && aligned(sg.grad_parts[r], u.grad_dtype == MFSDP_DTYPE_BF16 ? 8 : 16);
+                vec_parts16 = vec_parts16 && aligned(sg.grad_parts[r], 16);
             }
             for (int32_t d = 0; d < sg.ncopies; ++d) L.ptrs.push_back(reinterpret_cast<uint64_t>(sg.param_copies[d]));
         } else {
@@ -267,17 +270,50 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
         m.lda = round8(m.r);
         m.param_bf16 = u.param_dtype == MFSDP_DTYPE_BF16;
         m.grad_bf16 = u.grad_dtype == MFSDP_DTYPE_BF16;
-        m.mom_tile0 = tile0;
         m.mom_tiles_n = static_cast<int32_t>((u.cols + kMomTile - 1) / kMomTile);
         const int64_t tiles = ((u.rows + kMomTile - 1) / kMomTile) * m.mom_tiles_n;
         if (tile0 + tiles > (1LL << 31) - 1) return MFSDP_ERR_INVALID_ARG;
         tile0 += static_cast<int32_t>(tiles);
-        m.mom_grp0 = grp0;
-        grp0 += static_cast<int32_t>((tiles + kMomGroup - 1) / kMomGroup);
         m.mom_vec = (u.cols % 4 == 0) && aligned(u.momentum, 16) &&
                     (segs ? vec_parts : aligned(u.grad, u.grad_dtype == MFSDP_DTYPE_BF16 ? 8 : 16));
+        // flat runs: X = M (no transpose) with ldx == cols, and every access 16 bytes wide
+        bool flat = u.rows <= u.cols && u.cols % 8 == 0 && aligned(u.momentum, 16) && aligned(u.param, 16) &&
+                    (!u.update_out || aligned(u.update_out, 16)) && (segs ? vec_parts16 : aligned(u.grad, 16));
+        if (segs)
+            for (int32_t d = 0; d < segs[i].ncopies; ++d) flat = flat && aligned(segs[i].param_copies[d], 16);
+        m.mom_flat = flat ? 1 : 0;
+        const int64_t groups = flat ? (u.rows * u.cols + kFlatGroup - 1) / kFlatGroup
+                                    : (tiles + kMomGroup - 1) / kMomGroup;
+        if (grp0 + groups > (1LL << 31) - 1) return MFSDP_ERR_INVALID_ARG;
+        m.mom_groups_n = static_cast<int32_t>(groups);
+        grp0 += static_cast<int32_t>(groups);
         m.shape_scale = static_cast<float>(std::sqrt(std::max(1.0, static_cast<double>(u.rows) / u.cols)));
         L.mats.push_back(m);
+    }
+    // The streaming kernels run the flat matrices' groups and the tiled ones' in
+    // separate launches: order the records flat first (stable), then number the
+    // groups in that order, so that each launch covers one contiguous range.
+    {
+        std::vector<size_t> order(L.mats.size());
+        for (size_t k = 0; k < order.size(); ++k) order[k] = k;
+        std::stable_partition(order.begin(), order.end(), [&](size_t k) { return L.mats[k].mom_flat != 0; });
+        std::vector<MatDev> mats;
+        std::vector<size_t> firsts;
+        mats.reserve(order.size());
+        firsts.reserve(order.size());
+        for (size_t k : order) {
+            mats.push_back(L.mats[k]);
+            firsts.push_back(ptr_first[k]);
+        }
+        L.mats.swap(mats);
+        ptr_first.swap(firsts);
+        int32_t g = 0;
+        L.flat_groups = 0;
+        for (MatDev& m : L.mats) {
+            m.mom_grp0 = g;
+            g += m.mom_groups_n;
+            if (m.mom_flat) L.flat_groups = g;
+        }
     }
     L.mom_tiles = tile0;
     L.mom_groups = grp0;
@@ -304,15 +340,18 @@ int build_layout(const mfsdp_matrix* in, const mfsdp_owner_segments* segs, int32
     L.off_sym_seg = off;   off = align_up(off + seg_bytes);
     L.off_poly_seg = off;  off = align_up(off + seg_bytes);
     L.off_gen_seg = off;   off = align_up(off + seg_bytes);
-    L.off_partials = off;  off = align_up(off + static_cast<size_t>(L.mom_tiles) * sizeof(float));
+    L.off_partials = off;  off = align_up(off + static_cast<size_t>(L.mom_groups) * sizeof(float));
     L.off_s = off;         off = align_up(off + nm * sizeof(float));
     L.head_end = off;
     for (MatDev& m : L.mats) {
         const size_t x_elems = static_cast<size_t>(m.r) * m.ldx;
         const size_t a_elems = static_cast<size_t>(m.r) * m.lda;
+        // every region keeps at least kRegionSlack bytes after its end: a tensor-core
+        // operand load may read up to 126 bytes past a matrix's last valid element
+        // (values that only reach output columns the epilogue discards)
         auto take = [&](size_t bytes) -> char* {
             char* p = base ? base + off : nullptr;
-            off = align_up(off + bytes);
+            off = align_up(off + bytes + kRegionSlack);
             return p;
         };
         if (bf16) {
@@ -394,15 +433,33 @@ extern "C" int mfsdp_muon_step_launches(const mfsdp_matrix* mats, int32_t n, con
     if (!launches) return MFSDP_ERR_INVALID_ARG;
     int st = validate_all(mats, nullptr, n, hp);
     if (st) return st;
-    int32_t live = 0;
-    for (int32_t i = 0; i < n; ++i) live += (mats[i].rows > 0 && mats[i].cols > 0);
-    *launches = live == 0 ? 0 : 3 + 3 * hp->ns_steps;
+    Layout L;
+    st = build_layout(mats, nullptr, n, hp, nullptr, L, 1);
+    if (st) return st;
+    if (L.mats.empty()) {
+        *launches = 0;
+        return MFSDP_OK;
+    }
+    // momentum and parameter write: one launch each for the flat and the tiled matrices present
+    const int32_t streaming = (L.flat_groups > 0 ? 1 : 0) + (L.mom_groups > L.flat_groups ? 1 : 0);
+    *launches = 2 * streaming + 1 + 3 * hp->ns_steps;
     return MFSDP_OK;
 }
 
 extern "C" int mfsdp_muon_forget_workspace(void* workspace) {
     std::lock_guard<std::mutex> lock(g_cache_mu);
     g_cache.erase(reinterpret_cast<uintptr_t>(workspace));
+    return MFSDP_OK;
+}
+
+extern "C" int mfsdp_muon_forget_workspace_range(void* workspace, size_t bytes) {
+    const uintptr_t b = reinterpret_cast<uintptr_t>(workspace), e = b + bytes;
+    if (e < b) return MFSDP_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    for (auto it = g_cache.begin(); it != g_cache.end();) {
+        if (it->first >= b && it->first < e) it = g_cache.erase(it);
+        else ++it;
+    }
     return MFSDP_OK;
 }
 
@@ -416,6 +473,156 @@ extern "C" int mfsdp_muon_step_p2p(const mfsdp_matrix* mats, const mfsdp_owner_s
                                    void* stream) {
     if (n > 0 && !segs) return MFSDP_ERR_INVALID_ARG;
     return muon_step_impl(mats, segs, n, hp, workspace, workspace_bytes, stream);
+}
+
+namespace {
+
+constexpr int32_t kMaxOverlapGroups = 64;
+
+// Contiguous groups of about equal Newton-Schulz work, in list order: group k
+// ends at the first matrix where the running dense FLOP count reaches (k + 1) / G
+// of the total.  Returns G + 1 boundaries (empty groups dropped).
+std::vector<int32_t> overlap_bounds(const mfsdp_matrix* mats, int32_t n, int32_t groups) {
+    std::vector<double> cost(static_cast<size_t>(n), 0.0);
+    double total = 0.0;
+    for (int32_t i = 0; i < n; ++i) {
+        const double r = static_cast<double>(std::min(mats[i].rows, mats[i].cols));
+        const double c = static_cast<double>(std::max(mats[i].rows, mats[i].cols));
+        cost[i] = 4.0 * r * r * c + 2.0 * r * r * r;
+        total += cost[i];
+    }
+    std::vector<int32_t> b{0};
+    double acc = 0.0;
+    int32_t k = 1;
+    for (int32_t i = 0; i < n; ++i) {
+        acc += cost[i];
+        if (k < groups && acc >= total * k / groups && i + 1 < n) {
+            b.push_back(i + 1);
+            while (k < groups && acc >= total * k / groups) ++k;
+        }
+    }
+    b.push_back(n);
+    return b;
+}
+
+// The owner segments of one group with the copies left out (the copies of the
+// overlapped form move on the copy engines instead).
+std::vector<mfsdp_owner_segments> segs_without_copies(const mfsdp_owner_segments* segs, int32_t b0, int32_t b1) {
+    std::vector<mfsdp_owner_segments> out(segs + b0, segs + b1);
+    for (mfsdp_owner_segments& s : out) {
+        s.param_copies = nullptr;
+        s.ncopies = 0;
+    }
+    return out;
+}
+
+// Per-group workspace offsets (256-byte aligned) and the total.
+int overlap_workspace(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                      const mfsdp_muon_hparams* hp, const std::vector<int32_t>& b, std::vector<size_t>& off,
+                      std::vector<size_t>& bytes, size_t* total) {
+    off.clear();
+    bytes.clear();
+    size_t t = 0;
+    for (size_t g = 0; g + 1 < b.size(); ++g) {
+        const std::vector<mfsdp_owner_segments> gs = segs_without_copies(segs, b[g], b[g + 1]);
+        size_t sz = 0;
+        const int st = workspace_size_impl(mats + b[g], gs.data(), b[g + 1] - b[g], hp, &sz);
+        if (st) return st;
+        off.push_back(t);
+        bytes.push_back(sz);
+        t = align_up(t + sz);
+    }
+    *total = t;
+    return MFSDP_OK;
+}
+
+}  // namespace
+
+extern "C" int mfsdp_muon_workspace_size_p2p_overlap(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs,
+                                                     int32_t n, const mfsdp_muon_hparams* hp, int32_t groups,
+                                                     size_t* bytes) {
+    if (!bytes || groups < 1 || groups > kMaxOverlapGroups || (n > 0 && !segs)) return MFSDP_ERR_INVALID_ARG;
+    int st = validate_all(mats, segs, n, hp);
+    if (st) return st;
+    std::vector<size_t> off, sz;
+    return overlap_workspace(mats, segs, n, hp, overlap_bounds(mats, n, groups), off, sz, bytes);
+}
+
+extern "C" int mfsdp_muon_step_p2p_overlap(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
+                                           const mfsdp_muon_hparams* hp, int32_t groups, void* workspace,
+                                           size_t workspace_bytes, void* stream, void* copy_stream) {
+    if (groups < 1 || groups > kMaxOverlapGroups || (n > 0 && !segs)) return MFSDP_ERR_INVALID_ARG;
+    int st = validate_all(mats, segs, n, hp);
+    if (st) return st;
+    const std::vector<int32_t> b = overlap_bounds(mats, n, groups);
+    std::vector<size_t> off, sz;
+    size_t total = 0;
+    st = overlap_workspace(mats, segs, n, hp, b, off, sz, &total);
+    if (st) return st;
+    if (total == 0) return MFSDP_OK;
+    if (!workspace) return MFSDP_ERR_INVALID_ARG;
+    if (!aligned(workspace, kAlign)) return MFSDP_ERR_MISALIGNED;
+    if (workspace_bytes < total) return MFSDP_ERR_WORKSPACE_TOO_SMALL;
+    st = check_device();
+    if (st) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream), cs = static_cast<cudaStream_t>(copy_stream);
+    const size_t ngroups = b.size() - 1;
+    std::vector<cudaEvent_t> ev(ngroups + 1, nullptr);
+    auto release = [&]() {
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);   // released once the recorded work completes
+    };
+    for (cudaEvent_t& e : ev) {
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            release();
+            return MFSDP_ERR_CUDA;
+        }
+    }
+    char* base = static_cast<char*>(workspace);
+    bool any_copy = false;
+    for (size_t g = 0; g < ngroups; ++g) {
+        const int32_t b0 = b[g], b1 = b[g + 1];
+        const std::vector<mfsdp_owner_segments> gs = segs_without_copies(segs, b0, b1);
+        st = muon_step_impl(mats + b0, gs.data(), b1 - b0, hp, base + off[g], sz[g], stream);
+        if (st) {
+            release();
+            return st;
+        }
+        bool copies = false;
+        for (int32_t i = b0; i < b1; ++i) copies = copies || (segs[i].ncopies > 0 && mats[i].rows > 0 && mats[i].cols > 0);
+        if (!copies) continue;
+        any_copy = true;
+        // this group's parameters are final once its write kernel is done: move
+        // them on the copy engines while the next groups compute
+        if (cudaEventRecord(ev[g], s) != cudaSuccess || cudaStreamWaitEvent(cs, ev[g], 0) != cudaSuccess) {
+            cudaGetLastError();
+            release();
+            return MFSDP_ERR_CUDA;
+        }
+        for (int32_t i = b0; i < b1; ++i) {
+            const mfsdp_matrix& m = mats[i];
+            if (m.rows == 0 || m.cols == 0) continue;
+            const size_t nbytes = static_cast<size_t>(m.rows * m.cols) * (m.param_dtype == MFSDP_DTYPE_BF16 ? 2 : 4);
+            for (int32_t d = 0; d < segs[i].ncopies; ++d) {
+                if (cudaMemcpyAsync(segs[i].param_copies[d], m.param, nbytes, cudaMemcpyDefault, cs) != cudaSuccess) {
+                    cudaGetLastError();
+                    release();
+                    return MFSDP_ERR_CUDA;
+                }
+            }
+        }
+    }
+    if (any_copy) {
+        // the caller's stream completes only after every copy
+        if (cudaEventRecord(ev[ngroups], cs) != cudaSuccess || cudaStreamWaitEvent(s, ev[ngroups], 0) != cudaSuccess) {
+            cudaGetLastError();
+            release();
+            return MFSDP_ERR_CUDA;
+        }
+    }
+    release();
+    return MFSDP_OK;
 }
 
 int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* segs, int32_t n,
@@ -496,7 +703,7 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
     sc.bf16_mode = hp->mode == MFSDP_MODE_BF16;
 
     int slot = prof_before(MFSDP_KCLASS_MOMENTUM, s);
-    cudaError_t e = launch_momentum(d_mats, nm, L.mom_groups, sc, d_partials, segs != nullptr, s);
+    cudaError_t e = launch_momentum(d_mats, nm, L.flat_groups, L.mom_groups, sc, d_partials, segs != nullptr, s);
     prof_after(slot, s);
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     slot = prof_before(MFSDP_KCLASS_NORM, s);
@@ -531,7 +738,7 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
     // (iteration it reads copy it & 1 and writes the other)
     const int32_t xsel = hp->ns_steps & 1;
     slot = prof_before(MFSDP_KCLASS_WRITE, s);
-    e = launch_param_write(d_mats, nm, L.mom_groups, sc, d_s, xsel, hp->ns_steps == 0 ? 1 : 0, s);
+    e = launch_param_write(d_mats, nm, L.flat_groups, L.mom_groups, sc, d_s, xsel, hp->ns_steps == 0 ? 1 : 0, s);
     prof_after(slot, s);
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     return MFSDP_OK;

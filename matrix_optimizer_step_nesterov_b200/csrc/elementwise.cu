@@ -75,6 +75,39 @@ __device__ __forceinline__ float load1_master(const __nv_bfloat16* xb, const __n
     return master_value(__bfloat16_as_ushort(xb[i]), __bfloat16_as_ushort(xlo[i]));
 }
 
+// eight consecutive elements at p[i..i+7] as floats; i % 8 == 0 and p + i 16-byte aligned
+__device__ __forceinline__ void load8(const void* p, int64_t i, int bf16, float (&v)[8]) {
+    if (bf16) {
+        const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p) + i));
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            v[2 * k] = __uint_as_float(w[k] << 16);
+            v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+        }
+    } else {
+        const float4 a = __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(p) + i));
+        const float4 b = __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(p) + i) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+// bf16-mode master of X (master.cuh) at i..i+7, i % 8 == 0: one 16-byte store of each part
+__device__ __forceinline__ void store8_master(__nv_bfloat16* xb, __nv_bfloat16* xlo, int64_t i, const float (&v)[8]) {
+    uint32_t h[4], l[4];
+    #pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint16_t h0, l0, h1, l1;
+        master_split(v[2 * k], h0, l0);
+        master_split(v[2 * k + 1], h1, l1);
+        h[k] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+        l[k] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+    }
+    *reinterpret_cast<uint4*>(xb + i) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(xlo + i) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 // index of the matrix owning tile group `grp` (largest i with mom_grp0 <= grp)
 __device__ __forceinline__ int find_matrix(const MatDev* mats, int nmats, int grp) {
     int lo = 0, hi = nmats - 1;
@@ -100,6 +133,91 @@ __device__ __forceinline__ T block_sum(T v, T* smem) {
     return r;  // valid in thread 0
 }
 
+// Momentum over one flat group of an untransposed matrix: elements [e0, e0 + kFlatGroup)
+// of M (and of X, whose leading dimension is cols), in runs of 8 per thread, U runs
+// loaded before any arithmetic.  Returns this thread's sum of M^2.  GB: the gradient
+// is bf16 (else fp32; PARTS reads the owner-segment parts of either dtype).  U = 4 with
+// packed bf16 gradients; U = 2 otherwise.
+template <int U, bool PARTS, bool GB>
+__device__ __forceinline__ float momentum_flat(const MatDev& md, const StepScalars& sc, float* __restrict__ bufp,
+                                               const void* gradp, const void* const* parts, int nparts, int64_t e0,
+                                               int64_t n) {
+    const float beta = sc.beta, omb = 1.0f - sc.beta;
+    const int gbf = md.grad_bf16;
+    float* __restrict__ xf = md.xf[0];
+    __nv_bfloat16* __restrict__ xb = md.xb[0];
+    __nv_bfloat16* __restrict__ xl = md.xlo[0];
+    float sumsq = 0.f;
+    #pragma unroll 1
+    for (int c0 = 0; c0 < kFlatGroup / 8; c0 += U * 256) {
+        float4 bq[U][2];
+        uint4 gq[U][2];
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = e0 + 8 * (int64_t)(c0 + u * 256 + threadIdx.x);
+            if (i >= n) continue;
+            bq[u][0] = __ldcs(reinterpret_cast<const float4*>(bufp + i));
+            bq[u][1] = __ldcs(reinterpret_cast<const float4*>(bufp + i) + 1);
+            if (!PARTS) {
+                if (GB) {
+                    gq[u][0] = __ldcs(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(gradp) + i));
+                } else {
+                    gq[u][0] = __ldcs(reinterpret_cast<const uint4*>(static_cast<const float*>(gradp) + i));
+                    gq[u][1] = __ldcs(reinterpret_cast<const uint4*>(static_cast<const float*>(gradp) + i) + 1);
+                }
+            }
+        }
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = e0 + 8 * (int64_t)(c0 + u * 256 + threadIdx.x);
+            if (i >= n) continue;
+            float gv[8];
+            if (!PARTS) {
+                if (GB) {
+                    const uint32_t w[4] = {gq[u][0].x, gq[u][0].y, gq[u][0].z, gq[u][0].w};
+                    #pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        gv[2 * k] = __uint_as_float(w[k] << 16);
+                        gv[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+                    }
+                } else {
+                    const uint32_t w[8] = {gq[u][0].x, gq[u][0].y, gq[u][0].z, gq[u][0].w,
+                                           gq[u][1].x, gq[u][1].y, gq[u][1].z, gq[u][1].w};
+                    #pragma unroll
+                    for (int k = 0; k < 8; ++k) gv[k] = __uint_as_float(w[k]);
+                }
+            } else {
+                // the owner's gradient: contributions summed in rank order, in fp32
+                load8(parts[0], i, gbf, gv);
+                for (int r = 1; r < nparts; ++r) {
+                    float q[8];
+                    load8(parts[r], i, gbf, q);
+                    #pragma unroll
+                    for (int k = 0; k < 8; ++k) gv[k] += q[k];
+                }
+            }
+            const float bin[8] = {bq[u][0].x, bq[u][0].y, bq[u][0].z, bq[u][0].w,
+                                  bq[u][1].x, bq[u][1].y, bq[u][1].z, bq[u][1].w};
+            float bo[8], m[8];
+            #pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                bo[k] = beta * bin[k] + omb * gv[k];
+                m[k] = sc.nesterov ? omb * gv[k] + beta * bo[k] : bo[k];
+                sumsq += m[k] * m[k];
+            }
+            __stcs(reinterpret_cast<float4*>(bufp + i), make_float4(bo[0], bo[1], bo[2], bo[3]));
+            __stcs(reinterpret_cast<float4*>(bufp + i) + 1, make_float4(bo[4], bo[5], bo[6], bo[7]));
+            if (sc.bf16_mode) {
+                store8_master(xb, xl, i, m);
+            } else {
+                *reinterpret_cast<float4*>(xf + i) = make_float4(m[0], m[1], m[2], m[3]);
+                *reinterpret_cast<float4*>(xf + i + 4) = make_float4(m[4], m[5], m[6], m[7]);
+            }
+        }
+    }
+    return sumsq;
+}
+
 // ---------------------------------------------------------------------------
 // K1: one 64 x 64 tile of M per block of 256 threads.
 //   buf <- beta buf + (1-beta) G ;  M <- (1-beta) G + beta buf  (or M <- buf)
@@ -111,11 +229,11 @@ __device__ __forceinline__ T block_sum(T v, T* smem) {
 // ---------------------------------------------------------------------------
 template <bool PARTS>
 __global__ void __launch_bounds__(256, 4)
-momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
+momentum_kernel(const MatDev* __restrict__ mats, int nmats, int grp_base, StepScalars sc,
                 float* __restrict__ partials, int32_t* status) {
     __shared__ float tileM2[2][kMomTile][kMomTile + 1];
     __shared__ float red[8];
-    const int grp = blockIdx.x;
+    const int grp = grp_base + blockIdx.x;
     const int mi = find_matrix(mats, nmats, grp);
     const MatDev& md = mats[mi];
     const int64_t rows = md.rows, cols = md.cols;
@@ -251,6 +369,34 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     if (threadIdx.x == 0) partials[grp] = tot;
 }
 
+// K1 on flat matrices: one group (kFlatGroup contiguous elements of M and X) per
+// block of 256 threads, the group's sum of M^2 to partials[grp].  Three blocks
+// per SM leave each thread room for four runs of loads in flight.
+template <bool PARTS>
+__global__ void __launch_bounds__(256, 3)
+momentum_flat_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, float* __restrict__ partials,
+                     int32_t* status) {
+    __shared__ float red[8];
+    const int grp = blockIdx.x;
+    const int mi = find_matrix(mats, nmats, grp);
+    const MatDev& md = mats[mi];
+    if (grp < md.mom_grp0 || !md.mom_flat) {  // cannot happen with a host-built table
+        record_status(status, -7);
+        return;
+    }
+    const int64_t e0 = (int64_t)(grp - md.mom_grp0) * kFlatGroup;
+    const int64_t n = md.rows * md.cols;
+    float sumsq;
+    if (PARTS)
+        sumsq = momentum_flat<2, true, false>(md, sc, md.buf, md.grad, md.gparts, md.nparts, e0, n);
+    else if (md.grad_bf16)
+        sumsq = momentum_flat<4, false, true>(md, sc, md.buf, md.grad, md.gparts, md.nparts, e0, n);
+    else
+        sumsq = momentum_flat<2, false, false>(md, sc, md.buf, md.grad, md.gparts, md.nparts, e0, n);
+    const float tot = block_sum(sumsq, red);
+    if (threadIdx.x == 0) partials[grp] = tot;
+}
+
 // K2: s = 1 / (||M||_F + eps) per matrix; fixed-order fp64 sum of the group partials.
 __global__ void __launch_bounds__(256)
 norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict__ partials,
@@ -259,8 +405,7 @@ norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict_
     const int mi = blockIdx.x;
     if (mi >= nmats) return;
     const MatDev& md = mats[mi];
-    const int64_t tiles = ((md.rows + kMomTile - 1) / kMomTile) * md.mom_tiles_n;
-    const int64_t groups = (tiles + kMomGroup - 1) / kMomGroup;
+    const int64_t groups = md.mom_groups_n;
     double acc = 0.0;
     for (int64_t g = threadIdx.x; g < groups; g += blockDim.x) acc += (double)partials[md.mom_grp0 + g];
     const double tot = block_sum(acc, red);
@@ -275,11 +420,11 @@ norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict_
 // transposed X tile goes through shared memory so both X and W are read and
 // written along their rows; full tiles move 4 elements per access.
 __global__ void __launch_bounds__(256, 4)
-param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, const float* __restrict__ s,
-                   int xsel, int use_s, int32_t* status) {
+param_write_kernel(const MatDev* __restrict__ mats, int nmats, int grp_base, StepScalars sc,
+                   const float* __restrict__ s, int xsel, int use_s, int32_t* status) {
     // transposed tiles alternate between two staging tiles: one block barrier per tile
     __shared__ float tileX2[2][kMomTile][kMomTile + 1];
-    const int grp = blockIdx.x;
+    const int grp = grp_base + blockIdx.x;
     const int mi = find_matrix(mats, nmats, grp);
     const MatDev& md = mats[mi];
     const int64_t rows = md.rows, cols = md.cols;
@@ -312,6 +457,7 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
     bool wide = bfm && wbf && (cols % 8 == 0) && (reinterpret_cast<uintptr_t>(md.param) % 16 == 0) &&
                 (uo == nullptr || reinterpret_cast<uintptr_t>(uo) % 16 == 0);
     for (int d = 0; d < ncopies; ++d) wide = wide && (reinterpret_cast<uintptr_t>(copies[d]) % 16 == 0);
+
     for (int k = 0; k < kMomGroup; ++k) {
     const int local = (grp - grp0) * kMomGroup + k;
     if (local >= ntiles) break;      // block-uniform
@@ -471,6 +617,125 @@ param_write_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, c
     }
 }
 
+// The parameter write on flat matrices: one group (kFlatGroup contiguous elements
+// of W and X, the momentum kernel's groups) per block, runs of 8 elements, U runs
+// of raw loads in flight (bf16 values stay packed until used).
+//   BFM: X is the bf16 hi + lo master (else fp32);  WBF: W is bf16 (else fp32).
+template <int U, bool BFM, bool WBF>
+__device__ __forceinline__ void param_write_flat(const MatDev& md, const StepScalars& sc, float f,
+                                                 const float* __restrict__ xf, const __nv_bfloat16* __restrict__ xb,
+                                                 const __nv_bfloat16* __restrict__ xl, int64_t e0, int64_t n) {
+    const float lr = sc.lr, decay = sc.decay;
+    float* __restrict__ uo = md.update_out;
+    void* const* copies = md.pcopies;
+    const int ncopies = md.ncopies;
+    #pragma unroll 1
+    for (int c0 = 0; c0 < kFlatGroup / 8; c0 += U * 256) {
+        uint4 xq[U][2], wq[U][2];
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = e0 + 8 * (int64_t)(c0 + u * 256 + threadIdx.x);
+            if (i >= n) continue;
+            if (BFM) {
+                xq[u][0] = __ldcs(reinterpret_cast<const uint4*>(xb + i));
+                xq[u][1] = __ldcs(reinterpret_cast<const uint4*>(xl + i));
+            } else {
+                xq[u][0] = __ldcs(reinterpret_cast<const uint4*>(xf + i));
+                xq[u][1] = __ldcs(reinterpret_cast<const uint4*>(xf + i) + 1);
+            }
+            // W is written below: no streaming or read-only hint on its load
+            if (WBF) {
+                wq[u][0] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(md.param) + i);
+            } else {
+                wq[u][0] = *reinterpret_cast<const uint4*>(static_cast<const float*>(md.param) + i);
+                wq[u][1] = *(reinterpret_cast<const uint4*>(static_cast<const float*>(md.param) + i) + 1);
+            }
+        }
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = e0 + 8 * (int64_t)(c0 + u * 256 + threadIdx.x);
+            if (i >= n) continue;
+            float x[8], w[8];
+            const uint32_t a[4] = {xq[u][0].x, xq[u][0].y, xq[u][0].z, xq[u][0].w};
+            const uint32_t b[4] = {xq[u][1].x, xq[u][1].y, xq[u][1].z, xq[u][1].w};
+            #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (BFM) {
+                    x[2 * k] = master_value(static_cast<uint16_t>(a[k] & 0xFFFFu), static_cast<uint16_t>(b[k] & 0xFFFFu));
+                    x[2 * k + 1] = master_value(static_cast<uint16_t>(a[k] >> 16), static_cast<uint16_t>(b[k] >> 16));
+                } else {
+                    x[k] = __uint_as_float(a[k]);
+                    x[k + 4] = __uint_as_float(b[k]);
+                }
+            }
+            const uint32_t wa[4] = {wq[u][0].x, wq[u][0].y, wq[u][0].z, wq[u][0].w};
+            const uint32_t wb2[4] = {wq[u][1].x, wq[u][1].y, wq[u][1].z, wq[u][1].w};
+            #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (WBF) {
+                    w[2 * k] = __uint_as_float(wa[k] << 16);
+                    w[2 * k + 1] = __uint_as_float(wa[k] & 0xFFFF0000u);
+                } else {
+                    w[k] = __uint_as_float(wa[k]);
+                    w[k + 4] = __uint_as_float(wb2[k]);
+                }
+            }
+            float o[8];
+            #pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                o[k] = f * x[k];
+                w[k] = fmaf(-lr, o[k], w[k] * decay);
+            }
+            if (WBF) {
+                uint32_t nw[4];
+                #pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const __nv_bfloat162 p2 = __floats2bfloat162_rn(w[2 * k], w[2 * k + 1]);
+                    nw[k] = *reinterpret_cast<const uint32_t*>(&p2);
+                }
+                const uint4 out = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(md.param) + i) = out;
+                for (int d = 0; d < ncopies; ++d) *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(copies[d]) + i) = out;
+            } else {
+                const float4 lo = make_float4(w[0], w[1], w[2], w[3]), hi = make_float4(w[4], w[5], w[6], w[7]);
+                *reinterpret_cast<float4*>(static_cast<float*>(md.param) + i) = lo;
+                *(reinterpret_cast<float4*>(static_cast<float*>(md.param) + i) + 1) = hi;
+                for (int d = 0; d < ncopies; ++d) {
+                    *reinterpret_cast<float4*>(static_cast<float*>(copies[d]) + i) = lo;
+                    *(reinterpret_cast<float4*>(static_cast<float*>(copies[d]) + i) + 1) = hi;
+                }
+            }
+            if (uo) {
+                *reinterpret_cast<float4*>(uo + i) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4*>(uo + i + 4) = make_float4(o[4], o[5], o[6], o[7]);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256, 3)
+param_write_flat_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, const float* __restrict__ s,
+                        int xsel, int use_s, int32_t* status) {
+    const int grp = blockIdx.x;
+    const int mi = find_matrix(mats, nmats, grp);
+    const MatDev& md = mats[mi];
+    if (grp < md.mom_grp0 || !md.mom_flat) {  // cannot happen with a host-built table
+        record_status(status, -7);
+        return;
+    }
+    const int64_t e0 = (int64_t)(grp - md.mom_grp0) * kFlatGroup;
+    const int64_t n = md.rows * md.cols;
+    const float f = md.shape_scale * (use_s ? s[mi] : 1.0f);
+    const bool wbf = md.param_bf16 != 0;
+    if (sc.bf16_mode) {
+        if (wbf) param_write_flat<4, true, true>(md, sc, f, md.xf[xsel], md.xb[xsel], md.xlo[xsel], e0, n);
+        else param_write_flat<2, true, false>(md, sc, f, md.xf[xsel], md.xb[xsel], md.xlo[xsel], e0, n);
+    } else {
+        if (wbf) param_write_flat<2, false, true>(md, sc, f, md.xf[xsel], md.xb[xsel], md.xlo[xsel], e0, n);
+        else param_write_flat<2, false, false>(md, sc, f, md.xf[xsel], md.xb[xsel], md.xlo[xsel], e0, n);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // K6: AdamW over the packed fp32 tail.  28 algorithmic bytes per element.
 // ---------------------------------------------------------------------------
@@ -542,13 +807,23 @@ int sm_count() {
 
 }  // namespace
 
-cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_groups,
+cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t flat_groups, int32_t total_groups,
                             const StepScalars& sc, float* partials, bool parts, cudaStream_t st) {
-    if (total_groups <= 0) return cudaSuccess;
-    if (parts)
-        momentum_kernel<true><<<total_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
-    else
-        momentum_kernel<false><<<total_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
+    if (flat_groups > 0) {
+        if (parts)
+            momentum_flat_kernel<true><<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
+        else
+            momentum_flat_kernel<false><<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const int32_t tiled = total_groups - flat_groups;
+    if (tiled > 0) {
+        if (parts)
+            momentum_kernel<true><<<tiled, 256, 0, st>>>(d_mats, nmats, flat_groups, sc, partials, device_status_ptr());
+        else
+            momentum_kernel<false><<<tiled, 256, 0, st>>>(d_mats, nmats, flat_groups, sc, partials, device_status_ptr());
+    }
     return cudaGetLastError();
 }
 
@@ -559,10 +834,16 @@ cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partia
     return cudaGetLastError();
 }
 
-cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_groups, const StepScalars& sc,
-                               const float* s, int32_t xsel, int32_t use_s, cudaStream_t st) {
-    if (total_groups <= 0) return cudaSuccess;
-    param_write_kernel<<<total_groups, 256, 0, st>>>(d_mats, nmats, sc, s, xsel, use_s, device_status_ptr());
+cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t flat_groups, int32_t total_groups,
+                               const StepScalars& sc, const float* s, int32_t xsel, int32_t use_s, cudaStream_t st) {
+    if (flat_groups > 0) {
+        param_write_flat_kernel<<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, s, xsel, use_s, device_status_ptr());
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const int32_t tiled = total_groups - flat_groups;
+    if (tiled > 0)
+        param_write_kernel<<<tiled, 256, 0, st>>>(d_mats, nmats, flat_groups, sc, s, xsel, use_s, device_status_ptr());
     return cudaGetLastError();
 }
 

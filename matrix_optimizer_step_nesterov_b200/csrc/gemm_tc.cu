@@ -67,11 +67,11 @@ constexpr int kCtaGroup = 2;      // the engine's configuration
 // the diagonal tile is read through the transposed (MN-major) view of tile (J, I).
 struct alignas(64) TcMaps {
     CUtensorMap xk[2];   // X bf16 operand, K-major view: dims {c, r}, box {64, 128}
-    CUtensorMap xm[2];   // X bf16 operand, MN-major view: dims {c, r}, box {64, 64}
+    CUtensorMap xm[2];   // X bf16 operand, MN-major 3D view: dims {64, r, c/64}, box {64, 64, B_ROWS/64}
     CUtensorMap ea;      // E_A bf16, K-major view: dims {r, r}, box {64, 128}
     CUtensorMap eb;      // E_B bf16, K-major view: dims {r, r}, box {64, 128}
-    CUtensorMap eat;     // E_A bf16, MN-major view: dims {r, r}, box {64, 64}
-    CUtensorMap ebt;     // E_B bf16, MN-major view: dims {r, r}, box {64, 64}
+    CUtensorMap eat;     // E_A bf16, MN-major 3D view: dims {64, r, r/64}, box {64, 64, 2}
+    CUtensorMap ebt;     // E_B bf16, MN-major 3D view: dims {64, r, r/64}, box {64, 64, 2}
 };
 
 // ---------------------------------------------------------------------------
@@ -170,6 +170,21 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 3D tiled TMA loads (two 64-element MN chunks of an MN-major operand in one instruction)
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
+        : "memory");
 }
 
 // TMA load of this CTA's share of a cta_group::2 operand; completion is
@@ -626,16 +641,18 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                         if (CG == 2) tma_load_2d_pair(dst, map, fbl, x, y);
                         else tma_load_2d(dst, map, fbl, x, y);
                     };
+                    auto load3 = [&](uint32_t dst, const CUtensorMap* map, int chunk, int k) {
+                        if (CG == 2) tma_load_3d_pair(dst, map, fbl, 0, k, chunk);
+                        else tma_load_3d(dst, map, fbl, 0, k, chunk);
+                    };
                     if (a_t) {
-                        load(sa, amap_t, i0, kb * BK);               // A rows i0 .. i0 + 63, MN-major
-                        load(sa + BK * 128, amap_t, i0 + 64, kb * BK);
+                        load3(sa, amap_t, i0 / 64, kb * BK);         // A rows i0 .. i0 + 127, MN-major
                     } else {
                         load(sa, amap, kb * BK, i0);
                     }
                     if (gemm || b_t) {
                         const CUtensorMap* bm_ = gemm ? bmap : &mp.eat;
-                        #pragma unroll
-                        for (int q = 0; q < C::B_ROWS / 64; ++q) load(sb + q * (BK * 128), bm_, jb + 64 * q, kb * BK);
+                        load3(sb, bm_, jb / 64, kb * BK);            // B rows jb .. jb + B_ROWS - 1, MN-major
                     } else {
                         #pragma unroll
                         for (int h = 0; h < C::B_ROWS / 128; ++h) load(sb + h * (128 * BK * 2), bmap, kb * BK, jb + 128 * h);
@@ -822,6 +839,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// MN-major view for 3D loads: element (k, n) of a row-major [rows][ld] matrix as
+// (n % 64, k, n / 64); box {64, 64, chunks}.  The last chunk may run past column
+// `cols` (into the next row or the region's slack): those values only reach output
+// columns or rows past the matrix, which the epilogue discards.
+bool encode_3d_mn(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld_elems, uint32_t chunks) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, rows, (cols + 63) / 64};
+    const cuuint64_t strides[2] = {ld_elems * 2, 128};
+    const cuuint32_t box[3] = {64, 64, chunks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld_elems,
                uint32_t box_inner, uint32_t box_outer) {
     auto fn = encode_fn();
@@ -854,12 +887,12 @@ bool tc_encode_maps(const std::vector<MatDev>& mats, void* host_out) {
         TcMaps& mp = out[i];
         for (int b = 0; b < 2; ++b) {
             if (!encode_2d(&mp.xk[b], m.xb[b], m.c, m.r, m.ldx, BK, BM)) return false;
-            if (!encode_2d(&mp.xm[b], m.xb[b], m.c, m.r, m.ldx, 64, BK)) return false;
+            if (!encode_3d_mn(&mp.xm[b], m.xb[b], m.c, m.r, m.ldx, TcCfg<kCtaGroup>::B_ROWS / 64)) return false;
         }
         if (!encode_2d(&mp.ea, m.ab, m.r, m.r, m.lda, BK, BM)) return false;
         if (!encode_2d(&mp.eb, m.bm, m.r, m.r, m.lda, BK, BM)) return false;
-        if (!encode_2d(&mp.eat, m.ab, m.r, m.r, m.lda, 64, BK)) return false;
-        if (!encode_2d(&mp.ebt, m.bm, m.r, m.r, m.lda, 64, BK)) return false;
+        if (!encode_3d_mn(&mp.eat, m.ab, m.r, m.r, m.lda, 2)) return false;
+        if (!encode_3d_mn(&mp.ebt, m.bm, m.r, m.r, m.lda, 2)) return false;
     }
     return true;
 }

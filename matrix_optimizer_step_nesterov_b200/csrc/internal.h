@@ -33,11 +33,15 @@ struct MatDev {
     int32_t      tr;          // rows > cols
     int32_t      param_bf16;
     int32_t      grad_bf16;
-    int32_t      mom_tile0;   // first momentum tile of this matrix
+    int32_t      mom_flat;    // 1: the streaming kernels take this matrix as flat runs of
+                              //    kFlatGroup elements (untransposed, rows a multiple of 8
+                              //    elements, every user buffer 16-byte aligned); 0: as
+                              //    groups of kMomGroup 64 x 64 tiles
     int32_t      mom_tiles_n; // momentum tiles along cols
     int32_t      mom_vec;     // 1: 16-byte vector access is legal for this matrix
     float        shape_scale; // sqrt(max(1, rows/cols))
-    int32_t      mom_grp0;    // first tile group (kMomGroup tiles per block) of this matrix
+    int32_t      mom_grp0;    // first group (one block of the streaming kernels) of this matrix
+    int32_t      mom_groups_n;// groups of this matrix
     // owner-segment exchange (mfsdp_muon_step_p2p): the gradient is the fixed-order
     // sum of nparts contributions, and the updated parameter is also stored to
     // ncopies destinations; device arrays of pointers in the workspace head
@@ -83,6 +87,7 @@ struct StepScalars {
 
 constexpr int kMomTile = 64;   // momentum / parameter-write tile: 64 x 64 elements of M or W
 constexpr int kMomGroup = 4;   // tiles one block of those kernels processes
+constexpr int kFlatGroup = kMomGroup * kMomTile * kMomTile;   // elements of a flat group (16384)
 
 // The grouped step behind mfsdp_muon_step (segs == nullptr) and mfsdp_muon_step_p2p.
 // always_upload: enqueue the descriptor-table upload on every call instead of
@@ -101,14 +106,18 @@ int32_t* device_status_ptr();   // device address of this device's status word (
 
 // ---- launchers (return cudaError_t of the launch) ----
 // parts: the gradients are owner-segment sums (MatDev::gparts) rather than MatDev::grad
-cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t total_groups,
+// The streaming kernels run over groups: [0, flat_groups) belong to flat matrices
+// (a flat-run kernel), [flat_groups, total_groups) to tiled ones (a 64 x 64 tile
+// kernel); one launch each when non-empty.
+// parts: the gradients are owner-segment sums (MatDev::gparts) rather than MatDev::grad
+cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t flat_groups, int32_t total_groups,
                             const StepScalars& sc, float* partials, bool parts, cudaStream_t st);
 cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partials,
                         float* s_out, float eps, cudaStream_t st);
 // W <- W (1 - lr wd) - lr * scale * (use_s ? s : 1) * X, X from master copy xsel
 // (bf16 mode: xb[xsel] + xlo[xsel]; fp32 mode: xf[xsel])
-cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t total_groups, const StepScalars& sc,
-                               const float* s, int32_t xsel, int32_t use_s, cudaStream_t st);
+cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t flat_groups, int32_t total_groups,
+                               const StepScalars& sc, const float* s, int32_t xsel, int32_t use_s, cudaStream_t st);
 cudaError_t launch_gemm_simt(Phase ph, const MatDev* d_mats, int32_t nmats, const TileDev* d_tiles, int32_t ntiles,
                              int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st);
 cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, int64_t n,

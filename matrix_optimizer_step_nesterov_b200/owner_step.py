@@ -48,12 +48,16 @@ class MuonOwnerStep:
                  a: float = 3.4445, b: float = -4.7750, c: float = 2.0315, ns_steps: int = 5,
                  nesterov: bool = True, mode: str = "bf16",
                  grad_parts: Optional[Sequence[Sequence[torch.Tensor]]] = None,
-                 param_copies: Optional[Sequence[Sequence[torch.Tensor]]] = None):
+                 param_copies: Optional[Sequence[Sequence[torch.Tensor]]] = None,
+                 overlap_groups: int = 0):
         """``grad_parts[i]`` (optional): the ranks' contributions to matrix i's
         gradient, summed in order inside the step (``grads[i]`` may then be
         None); ``param_copies[i]``: tensors that receive the updated parameter.
         Either list turns the call into mfsdp_muon_step_p2p; the tensors may live
-        on peer GPUs that this device can access."""
+        on peer GPUs that this device can access.  ``overlap_groups`` > 0 runs
+        mfsdp_muon_step_p2p_overlap instead: the list in that many groups, each
+        group's copies on a side stream (the copy engines) while later groups
+        compute."""
         if not (len(params) == len(grads) == len(momenta)):
             raise ValueError("params, grads and momenta must have the same length")
         if update_outs is None:
@@ -92,11 +96,18 @@ class MuonOwnerStep:
         self.mats = mats
         self._arr = _lib.matrix_array(mats)
         self._segs = None
+        self.overlap_groups = int(overlap_groups)
+        if self.overlap_groups and not p2p:
+            raise ValueError("overlap_groups needs grad_parts or param_copies")
         if p2p:
             self._segs, self._seg_keep = _lib.owner_segments(
                 [[t.data_ptr() for t in parts] for parts in grad_parts],
                 [[t.data_ptr() for t in copies] for copies in param_copies])
-            self.workspace_bytes = _lib.mfsdp_muon_workspace_size_p2p(mats, self._segs, self.hp)
+            if self.overlap_groups:
+                self.workspace_bytes = _lib.mfsdp_muon_workspace_size_p2p_overlap(mats, self._segs, self.hp,
+                                                                                  self.overlap_groups)
+            else:
+                self.workspace_bytes = _lib.mfsdp_muon_workspace_size_p2p(mats, self._segs, self.hp)
         else:
             self.workspace_bytes = _lib.mfsdp_muon_workspace_size(mats, self.hp)
         dev = params[0].device if len(params) else torch.device("cuda")
@@ -105,9 +116,14 @@ class MuonOwnerStep:
         base = self._ws.data_ptr()
         self.workspace_ptr = (base + 255) // 256 * 256
         self.launches = _lib.mfsdp_muon_step_launches(mats, self.hp)
+        self._copy_stream = torch.cuda.Stream(device=dev) if self.overlap_groups else None
 
     def step(self, stream: Optional[torch.cuda.Stream] = None) -> None:
-        if self._segs is not None:
+        if self._segs is not None and self.overlap_groups:
+            _lib.mfsdp_muon_step_p2p_overlap(self.mats, self._segs, self.hp, self.overlap_groups,
+                                             self.workspace_ptr, self.workspace_bytes, _stream_handle(stream),
+                                             int(self._copy_stream.cuda_stream), arr=self._arr)
+        elif self._segs is not None:
             _lib.mfsdp_muon_step_p2p(self.mats, self._segs, self.hp, self.workspace_ptr, self.workspace_bytes,
                                      _stream_handle(stream), arr=self._arr)
         else:
@@ -126,7 +142,7 @@ class MuonOwnerStep:
 
     def close(self) -> None:
         if getattr(self, "_ws", None) is not None:
-            _lib.mfsdp_muon_forget_workspace(self.workspace_ptr)
+            _lib.mfsdp_muon_forget_workspace_range(self.workspace_ptr, max(self.workspace_bytes, 1))
             self._ws = None
 
     def __del__(self):

@@ -162,6 +162,9 @@ def test_launch_count(lib):
     assert lib.mfsdp_muon_step_launches([_mat(lib, 64, 64)], hp) == 3 + 3 * 5
     assert lib.mfsdp_muon_step_launches([_mat(lib, 64, 64)], lib.muon_hparams(ns_steps=0)) == 3
     assert lib.mfsdp_muon_step_launches([], hp) == 0
+    # a tall matrix is tiled, a wide one with 16-byte rows is flat: two streaming launches each
+    assert lib.mfsdp_muon_step_launches([_mat(lib, 128, 64), _mat(lib, 64, 128, base=1 << 30)], hp) == 5 + 3 * 5
+    assert lib.mfsdp_muon_step_launches([_mat(lib, 128, 64)], hp) == 3 + 3 * 5
 
 
 def test_adamw_validation(lib):
@@ -292,3 +295,21 @@ def test_tile_tables_cover_every_output_tile_once(lib):
             ms = mats if mode == lib.MFSDP_MODE_BF16 else [
                 lib.Matrix(m.param, m.grad, m.momentum, None, m.rows, m.cols, 0, 0) for m in mats]
             assert lib.mfsdp_muon_workspace_size(ms, lib.muon_hparams(mode=mode)) > 0, trial
+
+
+def test_overlap_entry_points_validate_and_size(lib):
+    hp = lib.muon_hparams()
+    mats = [_mat(lib, 256, 512), _mat(lib, 300, 100, base=1 << 30), _mat(lib, 128, 128, base=1 << 31)]
+    segs, keep = lib.owner_segments([[m.grad] for m in mats], [[(3 << 32) + (k << 24)] for k in range(len(mats))])
+    one = lib.mfsdp_muon_workspace_size_p2p(mats, segs, hp)
+    # one group: one region, the same size as the fused step's workspace
+    assert lib.mfsdp_muon_workspace_size_p2p_overlap(mats, segs, hp, 1) == one
+    # more groups: one region per group, each at least its own step's need
+    assert lib.mfsdp_muon_workspace_size_p2p_overlap(mats, segs, hp, 3) >= one
+    for bad in (0, 65):
+        with pytest.raises(lib.MfsdpError) as e:
+            lib.mfsdp_muon_workspace_size_p2p_overlap(mats, segs, hp, bad)
+        assert e.value.status == lib.MFSDP_ERR_INVALID_ARG
+    with pytest.raises(lib.MfsdpError) as e:
+        lib.mfsdp_muon_step_p2p_overlap(mats, segs, hp, 0, 0, 0, 0, 0)
+    assert e.value.status == lib.MFSDP_ERR_INVALID_ARG

@@ -115,3 +115,41 @@ def test_owner_update_equals_full_gradient_update(mode):
     Wb, Ob, Bb = run(False)
     for k in range(len(shapes)):
         assert torch.equal(Oa[k], Ob[k]) and torch.equal(Wa[k], Wb[k]) and torch.equal(Ba[k], Bb[k])
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+@pytest.mark.parametrize("groups", [1, 2, 3])
+def test_overlapped_materialisation_equals_the_fused_step(mode, groups):
+    """mfsdp_muon_step_p2p_overlap: the list in groups, each group's parameter
+    copies on a side stream while later groups compute; results bit for bit
+    those of the fused step, every copy equal to its parameter."""
+    from matrix_optimizer_step_nesterov_b200 import MuonOwnerStep
+    dtype = "bf16" if mode == "bf16" else "f32"
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    shapes = [(256, 512), (600, 300), (128, 128), (77, 1030), (512, 512)]
+    wl = custom_workload(shapes, dtype=dtype, seed=23)
+    hs = H.host_state(wl, wl.matrices, buf_init="random")
+    R, D = 2, 2
+    dev = torch.device("cuda")
+    parts = [split_grad(hs.G[k], R, 300 + k, dtype) for k in range(len(shapes))]
+
+    def run(overlap):
+        W = [torch.from_numpy(w).to(tdt).to(dev) for w in hs.W]
+        B = [torch.from_numpy(b).to(dev) for b in hs.buf]
+        O = [torch.empty(w.shape, dtype=torch.float32, device=dev) for w in W]
+        P = [[torch.from_numpy(p).to(tdt).to(dev) for p in parts[k]] for k in range(len(shapes))]
+        C = [[torch.full(w.shape, 3.0, dtype=tdt, device=dev) for _ in range(D)] for w in W]
+        st = MuonOwnerStep(W, [None] * len(W), B, O, mode=mode, grad_parts=P, param_copies=C,
+                           overlap_groups=overlap)
+        st.step()
+        st.step()
+        torch.cuda.synchronize()
+        st.close()
+        return W, O, B, C
+
+    Wf, Of, Bf, Cf = run(0)
+    Wo, Oo, Bo, Co = run(groups)
+    for k in range(len(shapes)):
+        assert torch.equal(Wf[k], Wo[k]) and torch.equal(Of[k], Oo[k]) and torch.equal(Bf[k], Bo[k])
+        for c in Co[k]:
+            assert torch.equal(c, Wo[k]), "a copy differs from its parameter"
