@@ -426,9 +426,16 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
         // column domain: the upper-triangle copies (row gi0 + rr < column gjc)
         const int gjc = gj0 + lane;
         if (interior) {
-            __nv_bfloat16* pu = ob + (int64_t)gi0 * lda + gjc;
+            // two adjacent columns per lane and two rows per instruction: 4-byte stores
+            const int cp = lane & 15, rp = lane >> 4;
+            uint32_t* pu = reinterpret_cast<uint32_t*>(ob + (int64_t)gi0 * lda + gj0) + cp;
+            const int64_t ldw = lda >> 1;             // lda is a multiple of 8
             #pragma unroll
-            for (int rr = 0; rr < 32; ++rr) pu[(int64_t)rr * lda] = __float2bfloat16_rn(stg[rr][lane]);
+            for (int k = 0; k < 16; ++k) {
+                const int rr = 2 * k + rp;
+                const __nv_bfloat162 v2 = __floats2bfloat162_rn(stg[rr][2 * cp], stg[rr][2 * cp + 1]);
+                pu[(int64_t)rr * ldw] = *reinterpret_cast<const uint32_t*>(&v2);
+            }
         } else {
             const bool col_ok = gjc < Ncols;
             #pragma unroll
@@ -442,60 +449,45 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
     }
 }
 
-// APPLY / FINAL input of half chunk b (16 rows of one 32-column chunk): the hi
-// and lo parts of X (master.cuh), copy `cur`, kept raw until used.  Lane l
-// takes the column pair 2 (l & 15), 2 (l & 15) + 1 of rows of parity l >> 4,
-// so each access moves a bf16 pair and a warp covers two rows of 32 columns.
-// (A pair may reach one column past the matrix: into the padding of the
-// leading dimension, which nothing reads.)
-__device__ __forceinline__ void x_load_half(const MatDev& md, int cur, int gi0, int gj_tile, int q0, int b,
-                                            int Mrows, int Ncols, int lane, uint32_t (&hv)[8], uint32_t (&lv)[8]) {
-    const uint32_t* xh = reinterpret_cast<const uint32_t*>(md.xb[cur]);
-    const uint32_t* xlo = reinterpret_cast<const uint32_t*>(md.xlo[cur]);
-    const int gjc = gj_tile + (q0 + (b >> 1)) * 32 + 2 * (lane & 15);
-    const int row0 = gi0 + (b & 1) * 16 + (lane >> 4);
-    const bool ok = gjc < Ncols;
-    const int64_t ldx = md.ldx;                    // even: a row is ldx / 2 pairs, two rows ldx pairs
-    const int64_t base = ((int64_t)row0 * ldx + gjc) >> 1;
-    if (gi0 + 32 <= Mrows && gj_tile + (q0 + (b >> 1)) * 32 + 32 <= Ncols) {   // warp-uniform: chunk inside X
-        #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            hv[k] = __ldg(xh + base + (int64_t)k * ldx);
-            lv[k] = __ldg(xlo + base + (int64_t)k * ldx);
-        }
-        return;
-    }
-    #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const bool in = ok && row0 + 2 * k < Mrows;
-        hv[k] = in ? __ldg(xh + base + (int64_t)k * ldx) : 0u;
-        lv[k] = in ? __ldg(xlo + base + (int64_t)k * ldx) : 0u;
+// APPLY / FINAL input of one quarter chunk (8 rows of a 32 x 32 chunk): the hi
+// and lo parts of X (master.cuh), copy `cur`, as 16-byte vectors.  Lane l takes
+// row `row` and the 8 columns from `col` = 8 (l & 3) of the chunk, so a warp
+// covers 8 rows of 32 columns.  (A vector may reach up to 7 columns past the
+// matrix: into the padding of the leading dimension, whose values only ever
+// reach discarded outputs.)
+__device__ __forceinline__ void x_load8(const MatDev& md, int cur, int row, int col, int Mrows, int Ncols, uint4& h,
+                                        uint4& l) {
+    if (row < Mrows && col < Ncols) {
+        const int64_t i = (int64_t)row * md.ldx + col;   // col and ldx multiples of 8: 16-byte aligned
+        h = __ldg(reinterpret_cast<const uint4*>(md.xb[cur] + i));
+        l = __ldg(reinterpret_cast<const uint4*>(md.xlo[cur] + i));
+    } else {
+        h = make_uint4(0u, 0u, 0u, 0u);
+        l = h;
     }
 }
 
 // APPLY / FINAL epilogue of one warp over its live chunks [q0, q1):
 //   X <- s ((a + d_B,i) X + E_B X)
 // X is read from copy iter & 1 (hi and lo parts, through the read-only path)
-// and written to the other copy; ch / cl hold the first half chunk, loaded by
-// the caller.
+// and written to the other copy, 8 elements (16 bytes of each part) per lane
+// and access; ch / cl hold the first quarter chunk, loaded by the caller.
 __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, const StepScalars& sc, float sg,
                                                 int gi0, int gj_tile, int q0, int q1, int Mrows, int Ncols,
-                                                uint32_t trow, float (*stg)[33], int lane, uint32_t (&ch)[8],
-                                                uint32_t (&cl)[8]) {
+                                                uint32_t trow, float (*stg)[33], int lane, uint4& ch, uint4& cl) {
     const int cur = iter & 1;
-    uint32_t* __restrict__ xhn = reinterpret_cast<uint32_t*>(md.xb[cur ^ 1]);
-    uint32_t* __restrict__ xlon = reinterpret_cast<uint32_t*>(md.xlo[cur ^ 1]);
+    __nv_bfloat16* __restrict__ xhn = md.xb[cur ^ 1];
+    __nv_bfloat16* __restrict__ xlon = md.xlo[cur ^ 1];
     const int64_t ldx = md.ldx;
     const int gi = gi0 + lane;
     const float fa = gi < Mrows ? (sc.a + __ldg(md.db + gi)) : 0.f;   // row domain: (a + d_B) of row gi
-    const int cp = lane & 15, rp = lane >> 4;
-    uint32_t nh[8], nl[8];
-    const int nb = 2 * (q1 - q0);                 // half-chunks of 16 rows
+    const int cq = lane & 3, r8 = lane >> 2;
+    const int nb = 4 * (q1 - q0);                 // quarter chunks of 8 rows
     #pragma unroll 1
     for (int b = 0; b < nb; ++b) {
-        const int q = q0 + (b >> 1);
-        const int h = (b & 1) * 16;
-        if (h == 0) {
+        const int q = q0 + (b >> 2);
+        const int k = b & 3;
+        if (k == 0) {
             uint32_t r[32];
             tmem_ld32(trow + q * 32, r);          // warp-collective
             __syncwarp();                         // previous chunk's reads of stg are done
@@ -503,31 +495,30 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
             for (int t = 0; t < 32; ++t) stg[lane][t] = __uint_as_float(r[t]);
             __syncwarp();
         }
-        if (b + 1 < nb) x_load_half(md, cur, gi0, gj_tile, q0, b + 1, Mrows, Ncols, lane, nh, nl);
-        const int gjc = gj_tile + q * 32 + 2 * cp;
-        const bool inside = gi0 + 32 <= Mrows && gj_tile + q * 32 + 32 <= Ncols;   // warp-uniform
-        #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int rr = h + rp + 2 * k;        // row within the chunk
-            const float fk = __shfl_sync(0xffffffffu, fa, rr);
-            if (inside || (gjc < Ncols && gi0 + rr < Mrows)) {
-                const float x0 = master_value(static_cast<uint16_t>(ch[k] & 0xFFFFu), static_cast<uint16_t>(cl[k] & 0xFFFFu));
-                const float x1 = master_value(static_cast<uint16_t>(ch[k] >> 16), static_cast<uint16_t>(cl[k] >> 16));
-                const float v0 = sg * fmaf(fk, x0, stg[rr][2 * cp]);
-                const float v1 = sg * fmaf(fk, x1, stg[rr][2 * cp + 1]);
-                uint16_t h0, l0, h1, l1;
-                master_split(v0, h0, l0);
-                master_split(v1, h1, l1);
-                const int64_t pidx = ((int64_t)(gi0 + rr) * ldx + gjc) >> 1;
-                xhn[pidx] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-                xlon[pidx] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+        uint4 nh, nl;
+        if (b + 1 < nb)
+            x_load8(md, cur, gi0 + r8 + 8 * ((b + 1) & 3), gj_tile + (q0 + ((b + 1) >> 2)) * 32 + 8 * cq, Mrows, Ncols,
+                    nh, nl);
+        const int rr = r8 + 8 * k;                // row within the chunk
+        const int col = gj_tile + q * 32 + 8 * cq;
+        const float fk = __shfl_sync(0xffffffffu, fa, rr);
+        if (gi0 + rr < Mrows && col < Ncols) {
+            const uint32_t hw[4] = {ch.x, ch.y, ch.z, ch.w}, lw[4] = {cl.x, cl.y, cl.z, cl.w};
+            uint32_t oh[4], ol[4];
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float x0 = master_value(static_cast<uint16_t>(hw[j] & 0xFFFFu), static_cast<uint16_t>(lw[j] & 0xFFFFu));
+                const float x1 = master_value(static_cast<uint16_t>(hw[j] >> 16), static_cast<uint16_t>(lw[j] >> 16));
+                const float v0 = sg * fmaf(fk, x0, stg[rr][8 * cq + 2 * j]);
+                const float v1 = sg * fmaf(fk, x1, stg[rr][8 * cq + 2 * j + 1]);
+                master_split2(v0, v1, oh[j], ol[j]);
             }
+            const int64_t i = (int64_t)(gi0 + rr) * ldx + col;
+            *reinterpret_cast<uint4*>(xhn + i) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+            *reinterpret_cast<uint4*>(xlon + i) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
         }
-        #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            ch[k] = nh[k];
-            cl[k] = nl[k];
-        }
+        ch = nh;
+        cl = nl;
     }
     __syncwarp();
 }
@@ -751,11 +742,12 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             const bool live = gi0 < Mrows && q0 < q1;
             // the first half chunk's inputs, loaded while the MMAs still run
             unsigned short pre_e[16];
-            uint32_t pre_h[8], pre_l[8];
+            uint4 pre_h, pre_l;
             float pre_dj = 0.f;
             if (live) {
                 if constexpr (gemm)
-                    x_load_half(md, iter & 1, gi0, gj_tile, q0, 0, Mrows, Ncols, lane, pre_h, pre_l);
+                    x_load8(md, iter & 1, gi0 + (lane >> 2), gj_tile + q0 * 32 + 8 * (lane & 3), Mrows, Ncols,
+                            pre_h, pre_l);
                 else
                     sym_load_half<ph>(md, td.tm != td.tn, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, lane, pre_e, pre_dj);
             }

@@ -22,6 +22,16 @@ __device__ __forceinline__ float master_value(uint16_t hi_bits, uint16_t lo_bits
     return bf16_bits_to_float(hi_bits) + bf16_bits_to_float(lo_bits);
 }
 
+// Two elements at once, packed as bf16 pairs (element 0 in the low half); each
+// element's parts are exactly those of master_split.
+__device__ __forceinline__ void master_split2(float x0, float x1, uint32_t& hi_pair, uint32_t& lo_pair) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    hi_pair = *reinterpret_cast<const uint32_t*>(&h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __uint_as_float(hi_pair << 16),
+                                                   x1 - __uint_as_float(hi_pair & 0xFFFF0000u));
+    lo_pair = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 __device__ __forceinline__ void master_split(float x, uint16_t& hi_bits, uint16_t& lo_bits) {
     hi_bits = __bfloat16_as_ushort(__float2bfloat16_rn(x));
     lo_bits = __bfloat16_as_ushort(__float2bfloat16_rn(x - bf16_bits_to_float(hi_bits)));
