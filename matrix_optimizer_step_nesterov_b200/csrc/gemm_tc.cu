@@ -591,6 +591,11 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
     if (CG == 2) cluster_sync();     // the peer's barriers are initialised before anyone signals them
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Programmatic dependent launch: the set-up above may overlap the previous
+    // phase's last tiles; nothing an earlier kernel wrote is read before this wait.
+    // The next phase may then launch as soon as every CTA of this one has started.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     constexpr bool gemm = (ph == PH_APPLY || ph == PH_FINAL);
     const int cur = iter & 1;
@@ -1038,8 +1043,11 @@ cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats
                          const int32_t* d_seg, int32_t clusters, int32_t iter, const StepScalars& sc, const float* s,
                          cudaStream_t st) {
     constexpr int CG = kCtaGroup;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = phase_config(clusters, st, attr);
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, tc_phase_kernel<ph, CG>, d_mats, maps, nmats, d_tiles, d_seg, iter, sc, s,
                               device_status_ptr());
 }
