@@ -703,7 +703,15 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
     sc.bf16_mode = hp->mode == MFSDP_MODE_BF16;
 
     int slot = prof_before(MFSDP_KCLASS_MOMENTUM, s);
-    cudaError_t e = launch_momentum(d_mats, nm, L.flat_groups, L.mom_groups, sc, d_partials, segs != nullptr, s);
+    // the flat groups stream through bulk copies when every flat matrix has the dtypes those kernels take
+    bool grads_bf16 = true, params_bf16 = true;
+    for (const MatDev& m : L.mats) {
+        if (!m.mom_flat) continue;
+        grads_bf16 = grads_bf16 && m.grad_bf16;
+        params_bf16 = params_bf16 && m.param_bf16;
+    }
+    cudaError_t e = launch_momentum(d_mats, nm, L.flat_groups, L.mom_groups, sc, d_partials, segs != nullptr,
+                                    grads_bf16, s);
     prof_after(slot, s);
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     slot = prof_before(MFSDP_KCLASS_NORM, s);
@@ -738,7 +746,8 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
     // (iteration it reads copy it & 1 and writes the other)
     const int32_t xsel = hp->ns_steps & 1;
     slot = prof_before(MFSDP_KCLASS_WRITE, s);
-    e = launch_param_write(d_mats, nm, L.flat_groups, L.mom_groups, sc, d_s, xsel, hp->ns_steps == 0 ? 1 : 0, s);
+    e = launch_param_write(d_mats, nm, L.flat_groups, L.mom_groups, sc, d_s, xsel, hp->ns_steps == 0 ? 1 : 0,
+                           params_bf16 && sc.bf16_mode, s);
     prof_after(slot, s);
     if (e != cudaSuccess) return MFSDP_ERR_CUDA;
     return MFSDP_OK;

@@ -397,6 +397,244 @@ momentum_flat_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc,
     if (threadIdx.x == 0) partials[grp] = tot;
 }
 
+// ---------------------------------------------------------------------------
+// Flat groups through 1D bulk copies (TMA): one thread streams a group's inputs
+// into a 3-stage shared-memory ring in runs of kBulkSub elements, the block
+// computes from shared memory and stores straight to global memory.  The
+// loads in flight cost no registers, so six blocks per SM keep up to 216 KB of
+// them in flight.  Every wait is bounded; on a timeout the block records
+// MFSDP_ERR_TIMEOUT, waits (bounded) for its own copies still in flight and
+// returns.
+// ---------------------------------------------------------------------------
+constexpr int kBulkSub = 2048;                  // elements per stage (one run of 8 per thread)
+constexpr int kBulkStages = 3;
+constexpr int kBulkSubs = kFlatGroup / kBulkSub;
+constexpr unsigned long long kBulkWaitNs = 1000000000ull;   // 1 s per wait
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void bulk_bar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void bulk_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// global -> shared, `bytes` a multiple of 16, both addresses 16-byte aligned
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool bulk_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(100000u)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long bulk_clock() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool bulk_wait(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
+    const unsigned long long t0 = bulk_clock();
+    while (!bulk_try_wait(bar, parity))
+        if (bulk_clock() - t0 > limit_ns) return false;
+    return true;
+}
+
+// The ring of one block: stage s of run k holds run k's slice of each input.
+// Thread 0 issues run k into stage k % kBulkStages once the block is done with
+// run k - kBulkStages; every thread waits for run k before using it.
+struct BulkRing {
+    uint64_t bar[kBulkStages];
+    int abort;
+};
+
+// Waits for run k (thread 0 polls, the block follows).  False on a timeout: the
+// block then drains (thread 0 waits, bounded, for the copies it issued) and stops.
+__device__ __forceinline__ bool bulk_ring_wait(BulkRing& ring, int k, int issued, int32_t* status) {
+    if (threadIdx.x == 0) {
+        const bool ok = bulk_wait(smem_u32(&ring.bar[k % kBulkStages]), (k / kBulkStages) & 1, kBulkWaitNs);
+        if (!ok) {
+            ring.abort = 1;
+            record_status(status, -6 /* MFSDP_ERR_TIMEOUT */);
+            for (int j = k; j < issued; ++j)   // the copies still in flight
+                (void)bulk_wait(smem_u32(&ring.bar[j % kBulkStages]), (j / kBulkStages) & 1, 10000000ull);
+        }
+    }
+    __syncthreads();
+    return ring.abort == 0;
+}
+
+// Momentum on one flat group with bf16 gradients (not the owner-segment sum).
+__global__ void __launch_bounds__(256)
+momentum_bulk_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, float* __restrict__ partials,
+                     int32_t* status) {
+    __shared__ __align__(128) float sbuf[kBulkStages][kBulkSub];
+    __shared__ __align__(128) __nv_bfloat16 sgrad[kBulkStages][kBulkSub];
+    __shared__ BulkRing ring;
+    __shared__ float red[8];
+    const int grp = blockIdx.x;
+    const int mi = find_matrix(mats, nmats, grp);
+    const MatDev& md = mats[mi];
+    if (grp < md.mom_grp0 || !md.mom_flat || !md.grad_bf16) {   // cannot happen with a host-built table
+        record_status(status, -7);
+        return;
+    }
+    const int64_t n = md.rows * md.cols;
+    const int64_t e0 = (int64_t)(grp - md.mom_grp0) * kFlatGroup;
+    const int64_t left = n - e0;                      // a multiple of 8, > 0
+    const int runs = static_cast<int>(min((int64_t)kBulkSubs, (left + kBulkSub - 1) / kBulkSub));
+    float* __restrict__ bufp = md.buf;
+    const __nv_bfloat16* gradp = static_cast<const __nv_bfloat16*>(md.grad);
+    auto issue = [&](int k) {                         // thread 0
+        const int64_t i0 = e0 + (int64_t)k * kBulkSub;
+        const uint32_t cnt = static_cast<uint32_t>(min((int64_t)kBulkSub, n - i0));
+        const uint32_t bar = smem_u32(&ring.bar[k % kBulkStages]);
+        bulk_expect(bar, cnt * 6);
+        bulk_load(smem_u32(sbuf[k % kBulkStages]), bufp + i0, cnt * 4, bar);
+        bulk_load(smem_u32(sgrad[k % kBulkStages]), gradp + i0, cnt * 2, bar);
+    };
+    int issued = 0;
+    if (threadIdx.x == 0) {
+        ring.abort = 0;
+        for (int s = 0; s < kBulkStages; ++s) bulk_bar_init(smem_u32(&ring.bar[s]));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (; issued < min(kBulkStages, runs); ++issued) issue(issued);
+    }
+    __syncthreads();
+    const float beta = sc.beta, omb = 1.0f - sc.beta;
+    float sumsq = 0.f;
+    for (int k = 0; k < runs; ++k) {
+        if (!bulk_ring_wait(ring, k, threadIdx.x == 0 ? issued : 0, status)) return;
+        const int st = k % kBulkStages;
+        const int64_t base = e0 + (int64_t)k * kBulkSub;
+        // two runs of 4 per thread, kBulkSub / 2 apart: conflict-free 16-byte shared reads
+        #pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int e = half * (kBulkSub / 2) + 4 * threadIdx.x;   // element within the stage
+            const int64_t i = base + e;
+            if (i >= n) continue;
+            const float4 b = *reinterpret_cast<const float4*>(&sbuf[st][e]);
+            const uint2 gq = *reinterpret_cast<const uint2*>(&sgrad[st][e]);
+            const float g[4] = {__uint_as_float(gq.x << 16), __uint_as_float(gq.x & 0xFFFF0000u),
+                                __uint_as_float(gq.y << 16), __uint_as_float(gq.y & 0xFFFF0000u)};
+            const float bin[4] = {b.x, b.y, b.z, b.w};
+            float bo[4], m[4];
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                bo[j] = beta * bin[j] + omb * g[j];
+                m[j] = sc.nesterov ? omb * g[j] + beta * bo[j] : bo[j];
+                sumsq += m[j] * m[j];
+            }
+            __stcs(reinterpret_cast<float4*>(bufp + i), make_float4(bo[0], bo[1], bo[2], bo[3]));
+            const float4 mv = make_float4(m[0], m[1], m[2], m[3]);
+            if (sc.bf16_mode) store4_master(md.xb[0], md.xlo[0], i, mv);
+            else *reinterpret_cast<float4*>(md.xf[0] + i) = mv;
+        }
+        __syncthreads();                              // every thread is done with stage st
+        if (threadIdx.x == 0 && issued < runs) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(issued++);
+        }
+    }
+    const float tot = block_sum(sumsq, red);
+    if (threadIdx.x == 0) partials[grp] = tot;
+}
+
+// The parameter write on one flat group, bf16 mode with a bf16 parameter.
+__global__ void __launch_bounds__(256)
+param_write_bulk_kernel(const MatDev* __restrict__ mats, int nmats, StepScalars sc, const float* __restrict__ s,
+                        int xsel, int use_s, int32_t* status) {
+    __shared__ __align__(128) __nv_bfloat16 sxh[kBulkStages][kBulkSub];
+    __shared__ __align__(128) __nv_bfloat16 sxl[kBulkStages][kBulkSub];
+    __shared__ __align__(128) __nv_bfloat16 sw[kBulkStages][kBulkSub];
+    __shared__ BulkRing ring;
+    const int grp = blockIdx.x;
+    const int mi = find_matrix(mats, nmats, grp);
+    const MatDev& md = mats[mi];
+    if (grp < md.mom_grp0 || !md.mom_flat || !md.param_bf16 || !sc.bf16_mode) {
+        record_status(status, -7);
+        return;
+    }
+    const int64_t n = md.rows * md.cols;
+    const int64_t e0 = (int64_t)(grp - md.mom_grp0) * kFlatGroup;
+    const int64_t left = n - e0;
+    const int runs = static_cast<int>(min((int64_t)kBulkSubs, (left + kBulkSub - 1) / kBulkSub));
+    const __nv_bfloat16* xh = md.xb[xsel];
+    const __nv_bfloat16* xl = md.xlo[xsel];
+    __nv_bfloat16* wp = static_cast<__nv_bfloat16*>(md.param);
+    auto issue = [&](int k) {
+        const int64_t i0 = e0 + (int64_t)k * kBulkSub;
+        const uint32_t cnt = static_cast<uint32_t>(min((int64_t)kBulkSub, n - i0));
+        const uint32_t bar = smem_u32(&ring.bar[k % kBulkStages]);
+        bulk_expect(bar, cnt * 6);
+        bulk_load(smem_u32(sxh[k % kBulkStages]), xh + i0, cnt * 2, bar);
+        bulk_load(smem_u32(sxl[k % kBulkStages]), xl + i0, cnt * 2, bar);
+        bulk_load(smem_u32(sw[k % kBulkStages]), wp + i0, cnt * 2, bar);
+    };
+    int issued = 0;
+    if (threadIdx.x == 0) {
+        ring.abort = 0;
+        for (int st = 0; st < kBulkStages; ++st) bulk_bar_init(smem_u32(&ring.bar[st]));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (; issued < min(kBulkStages, runs); ++issued) issue(issued);
+    }
+    __syncthreads();
+    const float f = md.shape_scale * (use_s ? s[mi] : 1.0f);
+    const float lr = sc.lr, decay = sc.decay;
+    float* __restrict__ uo = md.update_out;
+    void* const* copies = md.pcopies;
+    const int ncopies = md.ncopies;
+    for (int k = 0; k < runs; ++k) {
+        if (!bulk_ring_wait(ring, k, threadIdx.x == 0 ? issued : 0, status)) return;
+        const int st = k % kBulkStages;
+        const int64_t i = e0 + (int64_t)k * kBulkSub + 8 * threadIdx.x;
+        if (i < n) {
+            const uint4 h = reinterpret_cast<const uint4*>(sxh[st])[threadIdx.x];
+            const uint4 l = reinterpret_cast<const uint4*>(sxl[st])[threadIdx.x];
+            const uint4 wq = reinterpret_cast<const uint4*>(sw[st])[threadIdx.x];
+            const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+            const uint32_t ww[4] = {wq.x, wq.y, wq.z, wq.w};
+            float o[8];
+            uint32_t nw[4];
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                o[2 * j] = f * master_value(static_cast<uint16_t>(hw[j] & 0xFFFFu), static_cast<uint16_t>(lw[j] & 0xFFFFu));
+                o[2 * j + 1] = f * master_value(static_cast<uint16_t>(hw[j] >> 16), static_cast<uint16_t>(lw[j] >> 16));
+                const float w0 = __uint_as_float(ww[j] << 16), w1 = __uint_as_float(ww[j] & 0xFFFF0000u);
+                const __nv_bfloat162 p2 = __floats2bfloat162_rn(fmaf(-lr, o[2 * j], w0 * decay),
+                                                                fmaf(-lr, o[2 * j + 1], w1 * decay));
+                nw[j] = *reinterpret_cast<const uint32_t*>(&p2);
+            }
+            const uint4 out = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+            *reinterpret_cast<uint4*>(wp + i) = out;
+            for (int d = 0; d < ncopies; ++d) *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(copies[d]) + i) = out;
+            if (uo) {
+                *reinterpret_cast<float4*>(uo + i) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4*>(uo + i + 4) = make_float4(o[4], o[5], o[6], o[7]);
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0 && issued < runs) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(issued++);
+        }
+    }
+}
+
 // K2: s = 1 / (||M||_F + eps) per matrix; fixed-order fp64 sum of the group partials.
 __global__ void __launch_bounds__(256)
 norm_kernel(const MatDev* __restrict__ mats, int nmats, const float* __restrict__ partials,
@@ -808,10 +1046,12 @@ int sm_count() {
 }  // namespace
 
 cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t flat_groups, int32_t total_groups,
-                            const StepScalars& sc, float* partials, bool parts, cudaStream_t st) {
+                            const StepScalars& sc, float* partials, bool parts, bool flat_bulk, cudaStream_t st) {
     if (flat_groups > 0) {
         if (parts)
             momentum_flat_kernel<true><<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
+        else if (flat_bulk)
+            momentum_bulk_kernel<<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
         else
             momentum_flat_kernel<false><<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, partials, device_status_ptr());
         const cudaError_t e = cudaGetLastError();
@@ -835,9 +1075,13 @@ cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partia
 }
 
 cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t flat_groups, int32_t total_groups,
-                               const StepScalars& sc, const float* s, int32_t xsel, int32_t use_s, cudaStream_t st) {
+                               const StepScalars& sc, const float* s, int32_t xsel, int32_t use_s, bool flat_bulk,
+                               cudaStream_t st) {
     if (flat_groups > 0) {
-        param_write_flat_kernel<<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, s, xsel, use_s, device_status_ptr());
+        if (flat_bulk)
+            param_write_bulk_kernel<<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, s, xsel, use_s, device_status_ptr());
+        else
+            param_write_flat_kernel<<<flat_groups, 256, 0, st>>>(d_mats, nmats, sc, s, xsel, use_s, device_status_ptr());
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

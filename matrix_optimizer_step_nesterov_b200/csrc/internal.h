@@ -110,14 +110,17 @@ int32_t* device_status_ptr();   // device address of this device's status word (
 // (a flat-run kernel), [flat_groups, total_groups) to tiled ones (a 64 x 64 tile
 // kernel); one launch each when non-empty.
 // parts: the gradients are owner-segment sums (MatDev::gparts) rather than MatDev::grad
+// flat_bulk: every flat matrix has bf16 gradients (momentum) or a bf16 parameter in bf16
+// mode (parameter write), so its groups stream through 1D bulk copies
 cudaError_t launch_momentum(const MatDev* d_mats, int32_t nmats, int32_t flat_groups, int32_t total_groups,
-                            const StepScalars& sc, float* partials, bool parts, cudaStream_t st);
+                            const StepScalars& sc, float* partials, bool parts, bool flat_bulk, cudaStream_t st);
 cudaError_t launch_norm(const MatDev* d_mats, int32_t nmats, const float* partials,
                         float* s_out, float eps, cudaStream_t st);
 // W <- W (1 - lr wd) - lr * scale * (use_s ? s : 1) * X, X from master copy xsel
 // (bf16 mode: xb[xsel] + xlo[xsel]; fp32 mode: xf[xsel])
 cudaError_t launch_param_write(const MatDev* d_mats, int32_t nmats, int32_t flat_groups, int32_t total_groups,
-                               const StepScalars& sc, const float* s, int32_t xsel, int32_t use_s, cudaStream_t st);
+                               const StepScalars& sc, const float* s, int32_t xsel, int32_t use_s, bool flat_bulk,
+                               cudaStream_t st);
 cudaError_t launch_gemm_simt(Phase ph, const MatDev* d_mats, int32_t nmats, const TileDev* d_tiles, int32_t ntiles,
                              int32_t iter, const StepScalars& sc, const float* s, cudaStream_t st);
 cudaError_t launch_adamw(float* p, const float* g, float* m, float* v, int64_t n,
