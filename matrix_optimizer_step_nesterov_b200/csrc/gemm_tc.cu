@@ -467,14 +467,24 @@ __device__ __forceinline__ void x_load8(const MatDev& md, int cur, int row, int 
     }
 }
 
+// One whole chunk (its four quarters) of X for this lane: rows gi0 + (lane / 4) + 8k,
+// the 8 columns from col.
+__device__ __forceinline__ void x_load_chunk(const MatDev& md, int cur, int gi0, int col, int lane, int Mrows,
+                                             int Ncols, uint4 (&h)[4], uint4 (&l)[4]) {
+    #pragma unroll
+    for (int k = 0; k < 4; ++k) x_load8(md, cur, gi0 + (lane >> 2) + 8 * k, col, Mrows, Ncols, h[k], l[k]);
+}
+
 // APPLY / FINAL epilogue of one warp over its live chunks [q0, q1):
 //   X <- s ((a + d_B,i) X + E_B X)
 // X is read from copy iter & 1 (hi and lo parts, through the read-only path)
 // and written to the other copy, 8 elements (16 bytes of each part) per lane
-// and access; ch / cl hold the first quarter chunk, loaded by the caller.
+// and access.  The loads run a whole chunk ahead of their use (ch / cl hold
+// the first chunk, loaded by the caller while the MMAs still run).
 __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, const StepScalars& sc, float sg,
                                                 int gi0, int gj_tile, int q0, int q1, int Mrows, int Ncols,
-                                                uint32_t trow, float (*stg)[33], int lane, uint4& ch, uint4& cl) {
+                                                uint32_t trow, float (*stg)[33], int lane, uint4 (&ch)[4],
+                                                uint4 (&cl)[4]) {
     const int cur = iter & 1;
     __nv_bfloat16* __restrict__ xhn = md.xb[cur ^ 1];
     __nv_bfloat16* __restrict__ xlon = md.xlo[cur ^ 1];
@@ -482,43 +492,47 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
     const int gi = gi0 + lane;
     const float fa = gi < Mrows ? (sc.a + __ldg(md.db + gi)) : 0.f;   // row domain: (a + d_B) of row gi
     const int cq = lane & 3, r8 = lane >> 2;
-    const int nb = 4 * (q1 - q0);                 // quarter chunks of 8 rows
     #pragma unroll 1
-    for (int b = 0; b < nb; ++b) {
-        const int q = q0 + (b >> 2);
-        const int k = b & 3;
-        if (k == 0) {
-            uint32_t r[32];
-            tmem_ld32(trow + q * 32, r);          // warp-collective
-            __syncwarp();                         // previous chunk's reads of stg are done
+    for (int q = q0; q < q1; ++q) {
+        uint32_t r[32];
+        tmem_ld32(trow + q * 32, r);              // warp-collective
+        __syncwarp();                             // previous chunk's reads of stg are done
+        #pragma unroll
+        for (int t = 0; t < 32; ++t) stg[lane][t] = __uint_as_float(r[t]);
+        __syncwarp();
+        uint4 nh[4], nl[4];
+        if (q + 1 < q1) {
+            x_load_chunk(md, cur, gi0, gj_tile + (q + 1) * 32 + 8 * cq, lane, Mrows, Ncols, nh, nl);
+        } else {
             #pragma unroll
-            for (int t = 0; t < 32; ++t) stg[lane][t] = __uint_as_float(r[t]);
-            __syncwarp();
+            for (int k = 0; k < 4; ++k) nh[k] = nl[k] = make_uint4(0u, 0u, 0u, 0u);
         }
-        uint4 nh, nl;
-        if (b + 1 < nb)
-            x_load8(md, cur, gi0 + r8 + 8 * ((b + 1) & 3), gj_tile + (q0 + ((b + 1) >> 2)) * 32 + 8 * cq, Mrows, Ncols,
-                    nh, nl);
-        const int rr = r8 + 8 * k;                // row within the chunk
         const int col = gj_tile + q * 32 + 8 * cq;
-        const float fk = __shfl_sync(0xffffffffu, fa, rr);
-        if (gi0 + rr < Mrows && col < Ncols) {
-            const uint32_t hw[4] = {ch.x, ch.y, ch.z, ch.w}, lw[4] = {cl.x, cl.y, cl.z, cl.w};
-            uint32_t oh[4], ol[4];
-            #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float x0 = master_value(static_cast<uint16_t>(hw[j] & 0xFFFFu), static_cast<uint16_t>(lw[j] & 0xFFFFu));
-                const float x1 = master_value(static_cast<uint16_t>(hw[j] >> 16), static_cast<uint16_t>(lw[j] >> 16));
-                const float v0 = sg * fmaf(fk, x0, stg[rr][8 * cq + 2 * j]);
-                const float v1 = sg * fmaf(fk, x1, stg[rr][8 * cq + 2 * j + 1]);
-                master_split2(v0, v1, oh[j], ol[j]);
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int rr = r8 + 8 * k;            // row within the chunk
+            const float fk = __shfl_sync(0xffffffffu, fa, rr);
+            if (gi0 + rr < Mrows && col < Ncols) {
+                const uint32_t hw[4] = {ch[k].x, ch[k].y, ch[k].z, ch[k].w}, lw[4] = {cl[k].x, cl[k].y, cl[k].z, cl[k].w};
+                uint32_t oh[4], ol[4];
+                #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float x0 = master_value(static_cast<uint16_t>(hw[j] & 0xFFFFu), static_cast<uint16_t>(lw[j] & 0xFFFFu));
+                    const float x1 = master_value(static_cast<uint16_t>(hw[j] >> 16), static_cast<uint16_t>(lw[j] >> 16));
+                    const float v0 = sg * fmaf(fk, x0, stg[rr][8 * cq + 2 * j]);
+                    const float v1 = sg * fmaf(fk, x1, stg[rr][8 * cq + 2 * j + 1]);
+                    master_split2(v0, v1, oh[j], ol[j]);
+                }
+                const int64_t i = (int64_t)(gi0 + rr) * ldx + col;
+                *reinterpret_cast<uint4*>(xhn + i) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+                *reinterpret_cast<uint4*>(xlon + i) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
             }
-            const int64_t i = (int64_t)(gi0 + rr) * ldx + col;
-            *reinterpret_cast<uint4*>(xhn + i) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-            *reinterpret_cast<uint4*>(xlon + i) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
         }
-        ch = nh;
-        cl = nl;
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            ch[k] = nh[k];
+            cl[k] = nl[k];
+        }
     }
     __syncwarp();
 }
@@ -747,12 +761,12 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             const bool live = gi0 < Mrows && q0 < q1;
             // the first half chunk's inputs, loaded while the MMAs still run
             unsigned short pre_e[16];
-            uint4 pre_h, pre_l;
+            uint4 pre_h[4], pre_l[4];
             float pre_dj = 0.f;
             if (live) {
                 if constexpr (gemm)
-                    x_load8(md, iter & 1, gi0 + (lane >> 2), gj_tile + q0 * 32 + 8 * (lane & 3), Mrows, Ncols,
-                            pre_h, pre_l);
+                    x_load_chunk(md, iter & 1, gi0, gj_tile + q0 * 32 + 8 * (lane & 3), lane, Mrows, Ncols,
+                                 pre_h, pre_l);
                 else
                     sym_load_half<ph>(md, td.tm != td.tn, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, lane, pre_e, pre_dj);
             }
