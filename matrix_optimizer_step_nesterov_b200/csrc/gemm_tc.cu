@@ -644,8 +644,12 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                     const int kt = kb / (BN / BK);
                     const bool a_t = kSymA<ph> && kt < td.tm;
                     const bool b_t = kSymB<ph> && kt < td.tn;
-                    if (CG == 1) mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                    else if (leader) mbar_arrive_expect_tx(fb, CG * STAGE_BYTES);   // both CTAs' bytes
+                    // a diagonal tile of GRAM or POLY: this CTA's B rows are its A rows, in the
+                    // same view, so B is not loaded and the MMA reads it from the A buffer
+                    const bool diag = !gemm && td.tm == td.tn;
+                    const uint32_t bytes = diag ? A_BYTES : STAGE_BYTES;
+                    if (CG == 1) mbar_arrive_expect_tx(fb, bytes);
+                    else if (leader) mbar_arrive_expect_tx(fb, CG * bytes);   // both CTAs' bytes
                     const uint32_t fbl = (CG == 2) ? map_to_rank(fb, 0) : fb;
                     auto load = [&](uint32_t dst, const CUtensorMap* map, int x, int y) {
                         if (CG == 2) tma_load_2d_pair(dst, map, fbl, x, y);
@@ -660,7 +664,9 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                     } else {
                         load(sa, amap, kb * BK, i0);
                     }
-                    if (gemm || b_t) {
+                    if (diag) {
+                        // B comes from the A buffer (see above)
+                    } else if (gemm || b_t) {
                         const CUtensorMap* bm_ = gemm ? bmap : &mp.eat;
                         load3(sb, bm_, jb / 64, kb * BK);            // B rows jb .. jb + B_ROWS - 1, MN-major
                     } else {
@@ -702,7 +708,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                     if (!wait_bounded(full0 + 8 * stage, phase, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint32_t sb = sa + A_BYTES;
+                    const uint32_t sb = (!gemm && td.tm == td.tn) ? sa : sa + A_BYTES;   // the producer's diagonal case
                     const int kt = kb / (BN / BK);
                     const bool a_t = kSymA<ph> && kt < td.tm;           // same choice as the producer's
                     const bool b_t = gemm || (kSymB<ph> && kt < td.tn);
