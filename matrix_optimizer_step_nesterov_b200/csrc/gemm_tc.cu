@@ -43,7 +43,9 @@ constexpr int A_BYTES = BM * BK * 2;            // 16 KiB per CTA per stage
 constexpr int TMEM_COLS = 2 * BN;               // two fp32 accumulators
 constexpr int NUM_EPI_WARPS = 8;                // two per TMEM lane quadrant, each half the columns
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
-constexpr int STG_BYTES = NUM_EPI_WARPS * 32 * 33 * 4;   // epilogue staging: one 32 x 33 fp32 buffer per epilogue warp
+// epilogue staging, one 32 x 33-word buffer per epilogue warp: fp32 accumulators (APPLY,
+// FINAL) or, in its first 32 x 20 words, bf16 result pairs (GRAM, POLY)
+constexpr int STG_BYTES = NUM_EPI_WARPS * 32 * 33 * 4;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr uint32_t kSuspendHintNs = 200000u;                // one suspended try_wait: at most ~0.2 ms
 
@@ -292,19 +294,19 @@ __host__ __device__ constexpr uint32_t make_idesc(bool a_mn_major, bool b_mn_maj
 // ---------------------------------------------------------------------------
 
 // GRAM / POLY input of half chunk b of chunks [q0, ..): POLY's E_A(gi, gj) for
-// the 16 columns gj of the half, gj > gi.
+// the 16 columns gj of the half, gj > gi, and d_A of those 16 columns (the same
+// for every lane: broadcast loads).
 //   off-diagonal tile: the tile's own elements E_A[gi][gj], 16 consecutive
 //     elements of this lane's row (two 16-byte loads);
 //   diagonal tile: the mirrored elements E_A[gj][gi], consecutive across lanes
 //     (the diagonal tile is stored with both triangles).
 template <int ph>
 __device__ __forceinline__ void sym_load_half(const MatDev& md, bool offdiag, int gi, int gj_tile, int q0, int b,
-                                              int Mrows, int Ncols, int lane, unsigned short (&ev)[16], float& dj) {
+                                              int Mrows, int Ncols, unsigned short (&ev)[16], float4 (&dq)[4]) {
     if (ph != PH_POLY) return;
     const unsigned short* ab = reinterpret_cast<const unsigned short*>(md.ab);
     const int64_t lda = md.lda;
-    const int gj0 = gj_tile + (q0 + (b >> 1)) * 32;
-    const int gjh = gj0 + (b & 1) * 16;
+    const int gjh = gj_tile + (q0 + (b >> 1)) * 32 + (b & 1) * 16;
     const bool row_ok = gi < Mrows;
     if (offdiag) {
         if (row_ok && gjh + 16 <= Ncols) {
@@ -330,7 +332,22 @@ __device__ __forceinline__ void sym_load_half(const MatDev& md, bool offdiag, in
             ev[k] = (row_ok && gj < Ncols && gi < gj) ? __ldg(ab + (int64_t)gj * lda + gi) : (unsigned short)0;
         }
     }
-    if ((b & 1) == 0) dj = (gj0 + lane < Ncols) ? __ldg(md.da + gj0 + lane) : 0.f;   // d_A of column gj0 + lane
+    if (gjh + 16 <= Ncols) {
+        const float4* p = reinterpret_cast<const float4*>(md.da + gjh);   // 16-byte aligned (gjh % 16 == 0)
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) dq[k] = __ldg(p + k);
+    } else {
+        float d[16];
+        #pragma unroll
+        for (int k = 0; k < 16; ++k) d[k] = (gjh + k < Ncols) ? __ldg(md.da + gjh + k) : 0.f;
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) dq[k] = make_float4(d[4 * k], d[4 * k + 1], d[4 * k + 2], d[4 * k + 3]);
+    }
+}
+
+__device__ __forceinline__ float f4_elem(const float4 (&q)[4], int k) {
+    const float4 v = q[k >> 2];
+    return (k & 3) == 0 ? v.x : (k & 3) == 1 ? v.y : (k & 3) == 2 ? v.z : v.w;
 }
 
 // GRAM / POLY epilogue of one warp over its live chunks [q0, q1):
@@ -339,13 +356,17 @@ __device__ __forceinline__ void sym_load_half(const MatDev& md, bool offdiag, in
 //         ->  E_B (bf16), d_B
 // Results are stored block-upper: an off-diagonal tile (I < J) writes only
 // itself; a diagonal tile writes its upper triangle and mirrors it into its
-// lower triangle.  ev / dj hold the first half chunk's inputs, loaded by the
-// caller.
+// lower triangle.  The row-domain values go to the warp's staging buffer as the
+// bf16 pairs the column-domain stores write (32 rows of 20 words: 16 pairs and
+// 4 words of padding, so 16-byte writes and 4-byte reads are conflict-free).
+// ev / dq hold the first half chunk's inputs, loaded by the caller.
 template <int ph>
 __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepScalars& sc, float sg, bool offdiag,
                                                   int gi0, int gj_tile, int q0, int q1, int Mrows, int Ncols,
                                                   uint32_t trow, float (*stg)[33], int lane, unsigned short (&ev)[16],
-                                                  float dj) {
+                                                  float4 (&dq)[4]) {
+    constexpr int kSw = 20;                 // staging words per row
+    uint32_t* sb = reinterpret_cast<uint32_t*>(&stg[0][0]);   // [32][kSw] words (2560 bytes of the 4224)
     const int gi = gi0 + lane;      // row domain: this lane's row
     const bool row_ok = gi < Mrows;
     const int64_t lda = md.lda;
@@ -353,58 +374,47 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
     const float di = (ph == PH_POLY && row_ok) ? __ldg(md.da + gi) : 0.f;
     const float s2 = sg * sg;
     unsigned short en[16];
-    float djn = dj;
+    float4 dqn[4];
     const int nb = 2 * (q1 - q0);
     #pragma unroll 1
     for (int q = q0; q < q1; ++q) {
         const int gj0 = gj_tile + q * 32;
         uint32_t r[32];
         tmem_ld32(trow + q * 32, r);              // warp-collective
-        dj = djn;
         // warp-uniform: the whole 32 x 32 chunk is inside the matrix and strictly above the diagonal
         const bool interior = gi0 + 31 < Mrows && gj0 + 31 < Ncols && gi0 + 31 < gj0;
         #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {          // the chunk's two halves (h known at compile time)
             const int h = hh * 16;
             const int b = 2 * (q - q0) + hh;
-            if (b + 1 < nb) sym_load_half<ph>(md, offdiag, gi, gj_tile, q0, b + 1, Mrows, Ncols, lane, en, djn);
-            if (interior) {
-                // every element of the chunk lies strictly above the diagonal, inside the matrix
-                __nv_bfloat16* pm = ob + (int64_t)(gj0 + h) * lda + gi;   // E[gj][gi], gj = gj0 + h + k
-                #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int t = h + k;
-                    const float acc = __uint_as_float(r[t]);
-                    float val;
-                    if (ph == PH_GRAM) {
-                        val = s2 * acc;
-                    } else {
-                        const float dt = __shfl_sync(0xffffffffu, dj, t);
-                        const float e = bf16_bits_to_float(ev[k]);
-                        val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
-                    }
-                    if (!offdiag) pm[(int64_t)k * lda] = __float2bfloat16_rn(val);   // mirror inside the diagonal tile
-                    stg[lane][t] = val;
+            if (b + 1 < nb) sym_load_half<ph>(md, offdiag, gi, gj_tile, q0, b + 1, Mrows, Ncols, en, dqn);
+            // element k of the half: its value, with the diagonal tile's mirror and the
+            // diagonal entries stored on the way; each bf16 pair is packed as soon as
+            // both of its values exist
+            auto elem_in = [&](int k) -> float {   // interior chunks: strictly above the diagonal, inside
+                const float acc = __uint_as_float(r[h + k]);
+                float v;
+                if (ph == PH_GRAM) {
+                    v = s2 * acc;
+                } else {
+                    const float e = bf16_bits_to_float(ev[k]);
+                    v = sc.b * e + sc.c * fmaf(di + f4_elem(dq, k), e, acc);
                 }
-                #pragma unroll
-                for (int k = 0; k < 16; ++k) ev[k] = en[k];
-                continue;
-            }
-            #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int t = h + k;
-                const int gj = gj0 + t;
-                const float acc = __uint_as_float(r[t]);
-                const float dt = (ph == PH_POLY) ? __shfl_sync(0xffffffffu, dj, t) : 0.f;   // d_A of column gj
-                float val = 0.f;
+                if (!offdiag) ob[(int64_t)(gj0 + h + k) * lda + gi] = __float2bfloat16_rn(v);   // mirror
+                return v;
+            };
+            auto elem_edge = [&](int k) -> float {
+                const float acc = __uint_as_float(r[h + k]);
+                const int gj = gj0 + h + k;
+                float v = 0.f;
                 if (row_ok && gj < Ncols && gi <= gj) {
                     if (ph == PH_GRAM) {
-                        val = s2 * acc;
+                        v = s2 * acc;
                         if (gi == gj) {
-                            md.da[gi] = val;
+                            md.da[gi] = v;
                             ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
                         } else if (!offdiag) {
-                            ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);   // lower triangle, along column gj
+                            ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(v);   // lower triangle, along column gj
                         }
                     } else {
                         if (gi == gj) {
@@ -412,15 +422,35 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
                             ob[(int64_t)gi * lda + gi] = __float2bfloat16_rn(0.f);
                         } else {
                             const float e = bf16_bits_to_float(ev[k]);
-                            val = sc.b * e + sc.c * fmaf(di + dt, e, acc);
-                            if (!offdiag) ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(val);
+                            v = sc.b * e + sc.c * fmaf(di + f4_elem(dq, k), e, acc);
+                            if (!offdiag) ob[(int64_t)gj * lda + gi] = __float2bfloat16_rn(v);
                         }
                     }
                 }
-                stg[lane][t] = val;
+                return v;
+            };
+            // each bf16 pair is packed as soon as both of its values exist
+            uint32_t pk[8];
+            if (interior) {
+                #pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(elem_in(2 * k), elem_in(2 * k + 1));
+                    pk[k] = *reinterpret_cast<const uint32_t*>(&v2);
+                }
+            } else {
+                #pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(elem_edge(2 * k), elem_edge(2 * k + 1));
+                    pk[k] = *reinterpret_cast<const uint32_t*>(&v2);
+                }
             }
+            uint4* srow = reinterpret_cast<uint4*>(sb + lane * kSw + hh * 8);
+            srow[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            srow[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             #pragma unroll
             for (int k = 0; k < 16; ++k) ev[k] = en[k];
+            #pragma unroll
+            for (int k = 0; k < 4; ++k) dq[k] = dqn[k];
         }
         __syncwarp();
         // column domain: the upper-triangle copies (row gi0 + rr < column gjc)
@@ -433,16 +463,15 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
             #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int rr = 2 * k + rp;
-                const __nv_bfloat162 v2 = __floats2bfloat162_rn(stg[rr][2 * cp], stg[rr][2 * cp + 1]);
-                pu[(int64_t)rr * ldw] = *reinterpret_cast<const uint32_t*>(&v2);
+                pu[(int64_t)rr * ldw] = sb[rr * kSw + cp];
             }
         } else {
             const bool col_ok = gjc < Ncols;
-            #pragma unroll
+            const __nv_bfloat16* sh = reinterpret_cast<const __nv_bfloat16*>(sb);   // element (rr, c) at rr * 2 kSw + c
+            #pragma unroll 1
             for (int rr = 0; rr < 32; ++rr) {
                 const int gi2 = gi0 + rr;
-                if (gi2 < Mrows && col_ok && gi2 < gjc)
-                    ob[(int64_t)gi2 * lda + gjc] = __float2bfloat16_rn(stg[rr][lane]);
+                if (gi2 < Mrows && col_ok && gi2 < gjc) ob[(int64_t)gi2 * lda + gjc] = sh[rr * 2 * kSw + lane];
             }
         }
         __syncwarp();
@@ -768,13 +797,13 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             // the first half chunk's inputs, loaded while the MMAs still run
             unsigned short pre_e[16];
             uint4 pre_h[4], pre_l[4];
-            float pre_dj = 0.f;
+            float4 pre_dq[4];
             if (live) {
                 if constexpr (gemm)
                     x_load_chunk(md, iter & 1, gi0, gj_tile + q0 * 32 + 8 * (lane & 3), lane, Mrows, Ncols,
                                  pre_h, pre_l);
                 else
-                    sym_load_half<ph>(md, td.tm != td.tn, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, lane, pre_e, pre_dj);
+                    sym_load_half<ph>(md, td.tm != td.tn, gi0 + lane, gj_tile, q0, 0, Mrows, Ncols, pre_e, pre_dq);
             }
             bool ok = true;
             if (lane == 0) ok = wait_bounded(tfull0 + 8 * acc, acc_phase, abort_flag, status);
@@ -790,7 +819,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                                     pre_l);
                 else
                     epilogue_sym_warp<ph>(md, sc, sg, td.tm != td.tn, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg,
-                                          lane, pre_e, pre_dj);
+                                          lane, pre_e, pre_dq);
             }
             tc_fence_before();
             __syncwarp();
