@@ -43,9 +43,11 @@ constexpr int A_BYTES = BM * BK * 2;            // 16 KiB per CTA per stage
 constexpr int TMEM_COLS = 2 * BN;               // two fp32 accumulators
 constexpr int NUM_EPI_WARPS = 8;                // two per TMEM lane quadrant, each half the columns
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
-// epilogue staging, one 32 x 33-word buffer per epilogue warp: fp32 accumulators (APPLY,
-// FINAL) or, in its first 32 x 20 words, bf16 result pairs (GRAM, POLY)
-constexpr int STG_BYTES = NUM_EPI_WARPS * 32 * 33 * 4;
+// epilogue staging, one 32 x kStgW-word buffer per epilogue warp: fp32 accumulators (APPLY,
+// FINAL; 36-word rows make 16-byte writes along a row and 16-byte reads of 8-column runs
+// conflict-free) or, in its first 32 x 20 words, bf16 result pairs (GRAM, POLY)
+constexpr int kStgW = 36;
+constexpr int STG_BYTES = NUM_EPI_WARPS * 32 * kStgW * 4;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr uint32_t kSuspendHintNs = 200000u;                // one suspended try_wait: at most ~0.2 ms
 
@@ -57,7 +59,7 @@ template <int CG>
 struct TcCfg {
     static constexpr int B_ROWS = BN / CG;                      // B rows (N) this CTA loads
     static constexpr int STAGE_BYTES = A_BYTES + B_ROWS * BK * 2;
-    static constexpr int STAGES = CG == 1 ? 4 : 6;
+    static constexpr int STAGES = CG == 1 ? 4 : 5;
     static constexpr int TILE_M = BM * CG;                      // rows of a tile
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
 };
@@ -363,7 +365,7 @@ __device__ __forceinline__ float f4_elem(const float4 (&q)[4], int k) {
 template <int ph>
 __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepScalars& sc, float sg, bool offdiag,
                                                   int gi0, int gj_tile, int q0, int q1, int Mrows, int Ncols,
-                                                  uint32_t trow, float (*stg)[33], int lane, unsigned short (&ev)[16],
+                                                  uint32_t trow, float (*stg)[kStgW], int lane, unsigned short (&ev)[16],
                                                   float4 (&dq)[4]) {
     constexpr int kSw = 20;                 // staging words per row
     uint32_t* sb = reinterpret_cast<uint32_t*>(&stg[0][0]);   // [32][kSw] words (2560 bytes of the 4224)
@@ -510,9 +512,10 @@ __device__ __forceinline__ void x_load_chunk(const MatDev& md, int cur, int gi0,
 // and written to the other copy, 8 elements (16 bytes of each part) per lane
 // and access.  The loads run a whole chunk ahead of their use (ch / cl hold
 // the first chunk, loaded by the caller while the MMAs still run).
+template <bool S0>   // the first iteration: the Frobenius scale s applies (sg = s); later ones skip the product
 __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, const StepScalars& sc, float sg,
                                                 int gi0, int gj_tile, int q0, int q1, int Mrows, int Ncols,
-                                                uint32_t trow, float (*stg)[33], int lane, uint4 (&ch)[4],
+                                                uint32_t trow, float (*stg)[kStgW], int lane, uint4 (&ch)[4],
                                                 uint4 (&cl)[4]) {
     const int cur = iter & 1;
     __nv_bfloat16* __restrict__ xhn = md.xb[cur ^ 1];
@@ -527,7 +530,9 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
         tmem_ld32(trow + q * 32, r);              // warp-collective
         __syncwarp();                             // previous chunk's reads of stg are done
         #pragma unroll
-        for (int t = 0; t < 32; ++t) stg[lane][t] = __uint_as_float(r[t]);
+        for (int t = 0; t < 32; t += 4)
+            *reinterpret_cast<float4*>(&stg[lane][t]) = make_float4(__uint_as_float(r[t]), __uint_as_float(r[t + 1]),
+                                                                    __uint_as_float(r[t + 2]), __uint_as_float(r[t + 3]));
         __syncwarp();
         uint4 nh[4], nl[4];
         if (q + 1 < q1) {
@@ -543,13 +548,16 @@ __device__ __forceinline__ void epilogue_x_warp(const MatDev& md, int iter, cons
             const float fk = __shfl_sync(0xffffffffu, fa, rr);
             if (gi0 + rr < Mrows && col < Ncols) {
                 const uint32_t hw[4] = {ch[k].x, ch[k].y, ch[k].z, ch[k].w}, lw[4] = {cl[k].x, cl[k].y, cl[k].z, cl[k].w};
+                const float4 a0 = *reinterpret_cast<const float4*>(&stg[rr][8 * cq]);
+                const float4 a1 = *reinterpret_cast<const float4*>(&stg[rr][8 * cq + 4]);
+                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
                 uint32_t oh[4], ol[4];
                 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const float x0 = master_value(static_cast<uint16_t>(hw[j] & 0xFFFFu), static_cast<uint16_t>(lw[j] & 0xFFFFu));
                     const float x1 = master_value(static_cast<uint16_t>(hw[j] >> 16), static_cast<uint16_t>(lw[j] >> 16));
-                    const float v0 = sg * fmaf(fk, x0, stg[rr][8 * cq + 2 * j]);
-                    const float v1 = sg * fmaf(fk, x1, stg[rr][8 * cq + 2 * j + 1]);
+                    const float v0 = S0 ? sg * fmaf(fk, x0, av[2 * j]) : fmaf(fk, x0, av[2 * j]);
+                    const float v1 = S0 ? sg * fmaf(fk, x1, av[2 * j + 1]) : fmaf(fk, x1, av[2 * j + 1]);
                     master_split2(v0, v1, oh[j], ol[j]);
                 }
                 const int64_t i = (int64_t)(gi0 + rr) * ldx + col;
@@ -582,10 +590,12 @@ constexpr bool kSymB = ph == PH_POLY;
 template <int ph, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps, int32_t nmats,
-                const TileDev* __restrict__ tiles, const int32_t* __restrict__ seg, int32_t iter, StepScalars sc,
-                const float* __restrict__ s, int32_t* status) {
+                const TileDev* __restrict__ tiles, const int32_t* __restrict__ seg, int32_t iter, int32_t ring,
+                StepScalars sc, const float* __restrict__ s, int32_t* status) {
     using C = TcCfg<CG>;
     constexpr int STAGES = C::STAGES;
+    // stages of the ring this launch cycles through (the host's choice, at most the STAGES allocated)
+    const int nst = (ring >= 2 && ring <= STAGES) ? ring : STAGES;
     constexpr int STAGE_BYTES = C::STAGE_BYTES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned stage ring (128 B swizzle atoms need 1024 B alignment)
@@ -703,7 +713,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                         for (int h = 0; h < C::B_ROWS / 128; ++h) load(sb + h * (128 * BK * 2), bmap, kb * BK, jb + 128 * h);
                     }
                     issued[stage] = static_cast<int>(phase);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (++stage == nst) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok && leader) {
@@ -756,7 +766,7 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
                     // stage free (in both CTAs) once these MMAs finish
                     if (CG == 2) tc_commit2_both(empty0 + 8 * stage);
                     else tc_commit(empty0 + 8 * stage);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (++stage == nst) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
                 // accumulator ready for the epilogue (of both CTAs)
@@ -812,11 +822,17 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             tc_fence_after();
             const float sg = (iter == 0) ? s[td.mat] : 1.0f;
             const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
-            float (*stg)[33] = reinterpret_cast<float (*)[33]>(stg_all + (warp - 2) * 32 * 33);
+            float (*stg)[kStgW] = reinterpret_cast<float (*)[kStgW]>(stg_all + (warp - 2) * 32 * kStgW);
             if (live) {
                 if constexpr (gemm)
-                    epilogue_x_warp(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane, pre_h,
-                                    pre_l);
+                {
+                    if (iter == 0)
+                        epilogue_x_warp<true>(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane,
+                                              pre_h, pre_l);
+                    else
+                        epilogue_x_warp<false>(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane,
+                                               pre_h, pre_l);
+                }
                 else
                     epilogue_sym_warp<ph>(md, sc, sg, td.tm != td.tn, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg,
                                           lane, pre_e, pre_dq);
@@ -1089,15 +1105,15 @@ int device_clusters() {
 
 template <int ph>
 cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats, const TileDev* d_tiles,
-                         const int32_t* d_seg, int32_t clusters, int32_t iter, const StepScalars& sc, const float* s,
-                         cudaStream_t st) {
+                         const int32_t* d_seg, int32_t clusters, int32_t iter, int32_t ring, const StepScalars& sc,
+                         const float* s, cudaStream_t st) {
     constexpr int CG = kCtaGroup;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = phase_config(clusters, st, attr);
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, tc_phase_kernel<ph, CG>, d_mats, maps, nmats, d_tiles, d_seg, iter, sc, s,
+    return cudaLaunchKernelEx(&cfg, tc_phase_kernel<ph, CG>, d_mats, maps, nmats, d_tiles, d_seg, iter, ring, sc, s,
                               device_status_ptr());
 }
 
@@ -1105,18 +1121,50 @@ cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats
 
 int tc_max_clusters() { return device_clusters(); }
 
+// The ring depth a phase launch cycles through.  While the launch's operands
+// stay resident in L2, four stages keep the MMAs fed, and fewer loads in flight
+// per SM load the L2 less (same box: the skew workload 107.3 -> 102.7 ms, the
+// 7B share 52.4 -> 52.1 ms against five).  An operand larger than L2 streams
+// from DRAM and takes the fifth stage's latency cover (32B share: GRAM 9.8 ->
+// 9.4 ms per step).  Operand bytes: X (r x c) for GRAM and APPLY / FINAL, E_A
+// (r x r) for POLY.
+int tc_ring_depth(Phase ph, const std::vector<MatDev>& mats) {
+    static std::atomic<int64_t> l2_cached[kMaxDevices];   // zero: unknown
+    int dev = 0;
+    int64_t l2 = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
+        l2 = l2_cached[dev].load(std::memory_order_acquire);
+        if (l2 <= 0) {
+            int v = 0;
+            if (cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) == cudaSuccess && v > 0) {
+                l2 = v;
+                l2_cached[dev].store(l2, std::memory_order_release);
+            }
+        }
+    }
+    cudaGetLastError();
+    constexpr int deep = TcCfg<kCtaGroup>::STAGES;
+    if (l2 <= 0) return deep;
+    int64_t most = 0;
+    for (const MatDev& m : mats) {
+        const int64_t bytes = static_cast<int64_t>(m.r) * (ph == PH_POLY ? m.r : m.c) * 2;
+        most = std::max(most, bytes);
+    }
+    return most > l2 ? deep : 4;
+}
+
 cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, int32_t nmats,
-                           const TileDev* d_tiles, const int32_t* d_seg, int32_t clusters, int32_t iter,
+                           const TileDev* d_tiles, const int32_t* d_seg, int32_t clusters, int32_t iter, int32_t ring,
                            const StepScalars& sc, const float* s, cudaStream_t st) {
     if (clusters <= 0) return cudaSuccess;
     if (device_clusters() <= 0) return cudaErrorInvalidConfiguration;   // attributes not set on this device
     const TcMaps* maps = static_cast<const TcMaps*>(d_maps);
     cudaError_t e;
     switch (ph) {
-        case PH_GRAM: e = launch_phase<PH_GRAM>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, sc, s, st); break;
-        case PH_POLY: e = launch_phase<PH_POLY>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, sc, s, st); break;
-        case PH_APPLY: e = launch_phase<PH_APPLY>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, sc, s, st); break;
-        default: e = launch_phase<PH_FINAL>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, sc, s, st); break;
+        case PH_GRAM: e = launch_phase<PH_GRAM>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, ring, sc, s, st); break;
+        case PH_POLY: e = launch_phase<PH_POLY>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, ring, sc, s, st); break;
+        case PH_APPLY: e = launch_phase<PH_APPLY>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, ring, sc, s, st); break;
+        default: e = launch_phase<PH_FINAL>(d_mats, maps, nmats, d_tiles, d_seg, clusters, iter, ring, sc, s, st); break;
     }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -38,8 +38,13 @@ int tc_tile_cols();
 cudaError_t launch_bounded_wait_selftest(unsigned long long limit_ns, cudaStream_t st);
 
 // one phase over the tiles of d_tiles, partitioned by d_seg over `clusters` clusters
+// ring: the stages of the operand ring the launch cycles through (tc_ring_depth)
 cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, int32_t nmats,
-                           const TileDev* d_tiles, const int32_t* d_seg, int32_t clusters, int32_t iter,
+                           const TileDev* d_tiles, const int32_t* d_seg, int32_t clusters, int32_t iter, int32_t ring,
                            const StepScalars& sc, const float* s, cudaStream_t st);
+
+// the ring depth for a phase over these matrices: 4 while every operand fits in
+// the device's L2, else all the stages the kernel allocates
+int tc_ring_depth(Phase ph, const std::vector<MatDev>& mats);
 
 }  // namespace mfsdp
