@@ -724,14 +724,17 @@ int mfsdp::muon_step_impl(const mfsdp_matrix* mats, const mfsdp_owner_segments* 
     const int32_t* d_poly_seg = reinterpret_cast<const int32_t*>(base + L.off_poly_seg);
     const int32_t* d_gen_seg = reinterpret_cast<const int32_t*>(base + L.off_gen_seg);
     auto clusters = [](const std::vector<int32_t>& seg) { return static_cast<int32_t>(seg.size()) - 1; };
-    const int32_t ring_x = L.engine == Engine::Tc ? tc_ring_depth(PH_GRAM, L.mats) : 0;     // GRAM, APPLY, FINAL
-    const int32_t ring_poly = L.engine == Engine::Tc ? tc_ring_depth(PH_POLY, L.mats) : 0;
+    const bool tc = L.engine == Engine::Tc;
+    const int32_t ring_gram = tc ? tc_ring_depth(PH_GRAM, L.mats, nsym, clusters(L.sym_seg)) : 0;
+    const int32_t ring_poly = tc ? tc_ring_depth(PH_POLY, L.mats, nsym, clusters(L.poly_seg)) : 0;
+    const int32_t ring_gen = tc ? tc_ring_depth(PH_APPLY, L.mats, ngen, clusters(L.gen_seg)) : 0;
     auto gemm = [&](Phase ph, const TileDev* tiles, int32_t ntiles, const int32_t* d_seg, int32_t nclus, int32_t it,
                     int cls) {
         const int sl = prof_before(cls, s);
         const cudaError_t r = L.engine == Engine::Tc
                                   ? launch_gemm_tc(ph, d_mats, d_maps, nm, tiles, d_seg, nclus, it,
-                                                   ph == PH_POLY ? ring_poly : ring_x, sc, d_s, s)
+                                                   ph == PH_GRAM ? ring_gram : ph == PH_POLY ? ring_poly : ring_gen,
+                                                   sc, d_s, s)
                                   : launch_gemm_simt(ph, d_mats, nm, tiles, ntiles, it, sc, d_s, s);
         prof_after(sl, s);
         return r;

@@ -1121,14 +1121,16 @@ cudaError_t launch_phase(const MatDev* d_mats, const TcMaps* maps, int32_t nmats
 
 int tc_max_clusters() { return device_clusters(); }
 
-// The ring depth a phase launch cycles through.  While the launch's operands
-// stay resident in L2, four stages keep the MMAs fed, and fewer loads in flight
-// per SM load the L2 less (same box: the skew workload 107.3 -> 102.7 ms, the
-// 7B share 52.4 -> 52.1 ms against five).  An operand larger than L2 streams
-// from DRAM and takes the fifth stage's latency cover (32B share: GRAM 9.8 ->
-// 9.4 ms per step).  Operand bytes: X (r x c) for GRAM and APPLY / FINAL, E_A
-// (r x r) for POLY.
-int tc_ring_depth(Phase ph, const std::vector<MatDev>& mats) {
+// The ring depth a phase launch cycles through.  Under the power cap (long
+// launches over operands resident in L2) four stages keep the MMAs fed, and
+// fewer loads in flight per SM load the L2 less; three starve them.  Five
+// stages pay where the mainloop needs more latency cover: an operand larger
+// than L2 streams from DRAM, and a launch of fewer than 16 tiles per cluster
+// ends before the power cap lowers the clock.  Operand bytes: X (r x c) for
+// GRAM and APPLY / FINAL, E_A (r x r) for POLY.  Same box, ring 3 / 4 / 5:
+// skew 109.4 / 104.7 / 109.3 ms, 7B share 56.5 / 52.0 / 52.0 ms; block 2.18 /
+// 2.00 / 1.94 ms; 32B share (its X, 283 MB, from DRAM) - / 35.1 / 34.3 ms.
+int tc_ring_depth(Phase ph, const std::vector<MatDev>& mats, int64_t tiles, int32_t clusters) {
     static std::atomic<int64_t> l2_cached[kMaxDevices];   // zero: unknown
     int dev = 0;
     int64_t l2 = 0;
@@ -1150,7 +1152,7 @@ int tc_ring_depth(Phase ph, const std::vector<MatDev>& mats) {
         const int64_t bytes = static_cast<int64_t>(m.r) * (ph == PH_POLY ? m.r : m.c) * 2;
         most = std::max(most, bytes);
     }
-    return most > l2 ? deep : 4;
+    return (most > l2 || tiles < 16 * static_cast<int64_t>(clusters)) ? deep : 4;
 }
 
 cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, int32_t nmats,

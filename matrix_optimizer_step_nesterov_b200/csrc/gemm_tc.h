@@ -43,8 +43,9 @@ cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, i
                            const TileDev* d_tiles, const int32_t* d_seg, int32_t clusters, int32_t iter, int32_t ring,
                            const StepScalars& sc, const float* s, cudaStream_t st);
 
-// the ring depth for a phase over these matrices: 4 while every operand fits in
-// the device's L2, else all the stages the kernel allocates
-int tc_ring_depth(Phase ph, const std::vector<MatDev>& mats);
+// the ring depth for a phase launch of `tiles` tiles over `clusters` clusters on
+// these matrices: 4 for a long launch whose operands fit in the device's L2, else
+// all the stages the kernel allocates
+int tc_ring_depth(Phase ph, const std::vector<MatDev>& mats, int64_t tiles, int32_t clusters);
 
 }  // namespace mfsdp
