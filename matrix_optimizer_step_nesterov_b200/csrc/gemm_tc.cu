@@ -1125,8 +1125,8 @@ int tc_max_clusters() { return device_clusters(); }
 // launches over operands resident in L2) four stages keep the MMAs fed, and
 // fewer loads in flight per SM load the L2 less; three starve them.  Five
 // stages pay where the mainloop needs more latency cover: an operand larger
-// than L2 streams from DRAM, and a launch of fewer than 16 tiles per cluster
-// ends before the power cap lowers the clock.  Operand bytes: X (r x c) for
+// than L2 streams from DRAM, and a GRAM or APPLY launch of fewer than 16 tiles
+// per cluster ends before the power cap lowers the clock.  Operand bytes: X (r x c) for
 // GRAM and APPLY / FINAL, E_A (r x r) for POLY.  Same box, ring 3 / 4 / 5:
 // skew 109.4 / 104.7 / 109.3 ms, 7B share 56.5 / 52.0 / 52.0 ms; block 2.18 /
 // 2.00 / 1.94 ms; 32B share (its X, 283 MB, from DRAM) - / 35.1 / 34.3 ms.
@@ -1152,7 +1152,9 @@ int tc_ring_depth(Phase ph, const std::vector<MatDev>& mats, int64_t tiles, int3
         const int64_t bytes = static_cast<int64_t>(m.r) * (ph == PH_POLY ? m.r : m.c) * 2;
         most = std::max(most, bytes);
     }
-    return (most > l2 || tiles < 16 * static_cast<int64_t>(clusters)) ? deep : 4;
+    // POLY's short launches keep four (block workload: POLY 0.425 -> 0.414 ms per step)
+    const bool short_launch = ph != PH_POLY && tiles < 16 * static_cast<int64_t>(clusters);
+    return (most > l2 || short_launch) ? deep : 4;
 }
 
 cudaError_t launch_gemm_tc(Phase ph, const MatDev* d_mats, const void* d_maps, int32_t nmats,
