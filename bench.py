@@ -92,10 +92,10 @@ def ns_flops_dense(specs, steps: int = 5) -> float:
 
 # Per-launch DRAM bytes of the GEMM phases at the 7B share, from ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum) on the 4-matrix case
-# 2 x 4096^2 + 4096x11008 + 11008x4096: GRAM 0.4926 GB x 6.544, POLY 0.1095 GB x 7.0,
-# APPLY 1.1751 GB x 6.544 (X's and A's element counts), averaged over 5 GRAM + 5 POLY
+# 2 x 4096^2 + 4096x11008 + 11008x4096: GRAM 0.4968 GB x 6.544, POLY 0.1116 GB x 7.0,
+# APPLY 1.2954 GB x 6.544 (X's and A's element counts), averaged over 5 GRAM + 5 POLY
 # + 5 APPLY/FINAL launches.
-GEMM_TRAFFIC_7B = round((5 * 0.4926e9 * 6.544 + 5 * 0.1095e9 * 7.0 + 5 * 1.1751e9 * 6.544) / 15)
+GEMM_TRAFFIC_7B = round((5 * 0.4968e9 * 6.544 + 5 * 0.1116e9 * 7.0 + 5 * 1.2954e9 * 6.544) / 15)
 
 
 def split_groups(specs, n_groups: int) -> List[List[int]]:
