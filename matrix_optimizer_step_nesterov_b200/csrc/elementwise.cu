@@ -265,6 +265,23 @@ momentum_kernel(const MatDev* __restrict__ mats, int nmats, int grp_base, StepSc
     const int64_t ldx = md.ldx;
 
     if (full && mom_vec) {
+        // the next tile's momentum and gradient lines into L2 (one thread per 128-byte line)
+        if (!PARTS && k + 1 < kMomGroup && local + 1 < ntiles) {
+            const int tin = (local + 1) / tiles_n, tjn = (local + 1) % tiles_n;
+            const int64_t in0 = (int64_t)tin * kMomTile, jn0 = (int64_t)tjn * kMomTile;
+            if (in0 + kMomTile <= rows && jn0 + kMomTile <= cols) {
+                #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int v = e * 256 + threadIdx.x;
+                    const int64_t pidx = (in0 + (v >> 4)) * cols + jn0 + (v & 15) * 4;
+                    if ((v & 7) == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(bufp + pidx));
+                    if ((v & (gbf ? 15 : 7)) == 0)
+                        asm volatile("prefetch.global.L2 [%0];"
+                                     ::"l"(gbf ? static_cast<const void*>(static_cast<const __nv_bfloat16*>(gradp) + pidx)
+                                               : static_cast<const void*>(static_cast<const float*>(gradp) + pidx)));
+                }
+            }
+        }
         // all eight 16-byte loads of this thread are issued before any store
         float4 b[4], g[4];
         int64_t idx[4];
