@@ -368,7 +368,7 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
                                                   uint32_t trow, float (*stg)[kStgW], int lane, unsigned short (&ev)[16],
                                                   float4 (&dq)[4]) {
     constexpr int kSw = 20;                 // staging words per row
-    uint32_t* sb = reinterpret_cast<uint32_t*>(&stg[0][0]);   // [32][kSw] words (2560 bytes of the 4224)
+    uint32_t* sb = reinterpret_cast<uint32_t*>(&stg[0][0]);   // [32][kSw] words (2560 of the buffer's 4608 bytes)
     const int gi = gi0 + lane;      // row domain: this lane's row
     const bool row_ok = gi < Mrows;
     const int64_t lda = md.lda;
@@ -391,8 +391,7 @@ __device__ __forceinline__ void epilogue_sym_warp(const MatDev& md, const StepSc
             const int b = 2 * (q - q0) + hh;
             if (b + 1 < nb) sym_load_half<ph>(md, offdiag, gi, gj_tile, q0, b + 1, Mrows, Ncols, en, dqn);
             // element k of the half: its value, with the diagonal tile's mirror and the
-            // diagonal entries stored on the way; each bf16 pair is packed as soon as
-            // both of its values exist
+            // diagonal entries stored on the way
             auto elem_in = [&](int k) -> float {   // interior chunks: strictly above the diagonal, inside
                 const float acc = __uint_as_float(r[h + k]);
                 float v;
