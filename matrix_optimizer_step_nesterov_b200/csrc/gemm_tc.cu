@@ -823,18 +823,17 @@ tc_phase_kernel(const MatDev* __restrict__ mats, const TcMaps* __restrict__ maps
             const uint32_t trow = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
             float (*stg)[kStgW] = reinterpret_cast<float (*)[kStgW]>(stg_all + (warp - 2) * 32 * kStgW);
             if (live) {
-                if constexpr (gemm)
-                {
+                if constexpr (gemm) {
                     if (iter == 0)
                         epilogue_x_warp<true>(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane,
                                               pre_h, pre_l);
                     else
                         epilogue_x_warp<false>(md, iter, sc, sg, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg, lane,
                                                pre_h, pre_l);
-                }
-                else
+                } else {
                     epilogue_sym_warp<ph>(md, sc, sg, td.tm != td.tn, gi0, gj_tile, q0, q1, Mrows, Ncols, trow, stg,
                                           lane, pre_e, pre_dq);
+                }
             }
             tc_fence_before();
             __syncwarp();
